@@ -1,0 +1,120 @@
+/*
+ * hv_attn.h - C ABI of the joint 3D-RoPE full-attention library (libhvattn.so).
+ *
+ * What it computes. For every batch sample b and head h, over the joint
+ * sequence [video tokens ; text tokens] (HunyuanVideo 模型结构与数学原理,
+ * §5.2 "双流块": Q=[Q_v;Q_t], K=[K_v;K_t], V=[V_v;V_t],
+ * Attn = softmax(QK^T/sqrt(128))V, joint length S = N + L):
+ *
+ *   q'_i = R(t_i,h_i,w_i) q_i for video rows i < N, q'_i = q_i for text rows;
+ *   k'_j likewise;                                     (§5.5 "3D RoPE")
+ *   out_i = sum_{j < N+valid_b} softmax_j(scale * q'_i . k'_j) v_j.
+ *
+ * R = R_t (+) R_h (+) R_w acts on the head dimension 128 split into
+ * (d_t, d_h, d_w) = (16, 56, 56) channel segments (§5.5; the tech-report
+ * summary's Table 2); inside a segment of width d, the adjacent channel pair
+ * (2i, 2i+1) turns by pos * theta^(-2i/d) as
+ * (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos), pos being the token's
+ * t, h or w coordinate. Video tokens are the T x Hp x Wp patch grid flattened
+ * t-major, then h, then w (token n: t = n/(Hp*Wp), h = (n/Wp)%Hp, w = n%Wp);
+ * text tokens are not rotated. Keys at or past N + text_valid[b] (text
+ * padding) are masked out; every query row, padded text rows included, is
+ * computed and written.
+ *
+ * All calls are plain C, return an hv_status code, never throw and never
+ * abort the process.
+ */
+#ifndef HV_ATTN_H
+#define HV_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum hv_status {
+    HV_OK = 0,
+    HV_ERR_NULL_POINTER = 1,   /* a required pointer is NULL                        */
+    HV_ERR_MISALIGNED = 2,     /* q/k/v/out not 16-byte aligned                      */
+    HV_ERR_BAD_SHAPE = 3,      /* B, heads, T, Hp or Wp < 1, or B > HV_MAX_BATCH     */
+    HV_ERR_BAD_TEXT = 4,       /* text_len not in [0,256] or text_valid[b] not in [0,text_len] */
+    HV_ERR_TOO_LARGE = 5,      /* S*heads*128 or a TMA coordinate exceeds int32      */
+    HV_ERR_ALIAS = 6,          /* out overlaps q, k or v                             */
+    HV_ERR_BAD_SCALAR = 7,     /* rope_theta <= 0 or not finite, scale not finite    */
+    HV_ERR_NO_DEVICE = 8,      /* current CUDA device is not an sm_100 (B200) part   */
+    HV_ERR_LAUNCH = 9,         /* a CUDA runtime/driver call failed                  */
+    HV_ERR_DEVICE_TIMEOUT = 10 /* a kernel-side wait ran out (see hv_attn_last_device_error) */
+};
+
+#define HV_HEAD_DIM 128
+#define HV_MAX_TEXT_LEN 256
+#define HV_MAX_BATCH 512
+
+/*
+ * hv_attn_forward - joint full self-attention with 3D RoPE on the video rows.
+ *
+ * q, k, v  : device pointers, bf16, layout [B, S, heads, 128] row-major and
+ *            contiguous (S = T*Hp*Wp + text_len; the last three dims
+ *            [S, heads, 128] as in §5.6 "用张量形状读一个 Transformer block"),
+ *            video tokens first, then text_len text tokens (valid first,
+ *            padding last). Un-rotated: the call applies the rotation.
+ *            Padded text rows of k and v must hold finite values (they get
+ *            probability 0, and 0 * NaN would still poison the sum).
+ * out      : device pointer, bf16, same layout; every row is written.
+ *            Must not overlap q, k or v.
+ * B, heads : batch and head count (>= 1, B <= HV_MAX_BATCH).
+ * T, Hp, Wp: video-token grid (T' = floor((F-1)/4)+1, Hp = H/16, Wp = W/16
+ *            for an F x H x W clip; see hv_video_tokens), each >= 1.
+ * text_len : text tokens per sample in the buffers, 0..256 (the MLLM branch
+ *            keeps at most 256 prompt tokens, §3.1).
+ * text_valid: HOST pointer to B ints, 0 <= text_valid[b] <= text_len; read
+ *            before the call returns (the caller may free it right after).
+ * rope_theta: RoPE base (> 0; the pages' default is 256).
+ * scale    : softmax scale (finite; the pages use 1/sqrt(128)).
+ * cuda_stream: cudaStream_t to enqueue on (NULL = legacy default stream).
+ *
+ * Ownership: the caller owns all buffers; the library allocates no device
+ * memory. Asynchronous: enqueues one kernel and returns without
+ * synchronising. Errors in the arguments are reported before anything is
+ * launched. A kernel-side wait that runs out (a broken pipeline, never an
+ * expected event) sets the device error word read by
+ * hv_attn_last_device_error; the kernel then ends cleanly.
+ */
+int hv_attn_forward(const void* q, const void* k, const void* v, void* out,
+                    int B, int heads, int T, int Hp, int Wp,
+                    int text_len, const int* text_valid,
+                    float rope_theta, float scale, void* cuda_stream);
+
+/*
+ * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)
+ * of an F x H x W clip (§4 "Causal 3D VAE": temporal compression 4 keeping the
+ * first frame, spatial 8, then the 1x2x2 patch). Returns -1 when F is not
+ * 4k+1 (k >= 0) or H, W are not positive multiples of 16. Pure host function.
+ */
+long long hv_video_tokens(int frames, int height, int width);
+
+/*
+ * hv_attn_last_device_error - synchronises the current device, returns the
+ * device-side error word accumulated by kernels of this library since the
+ * previous call, and clears it. 0 = none. Otherwise bit 0 is set for a wait
+ * that ran out, and bits 8..15 name the waiting role (1 producer, 2 MMA,
+ * 3 softmax, 4 RoPE, 5 self-test). Returns -1 if the device cannot be read.
+ */
+int hv_attn_last_device_error(void);
+
+/*
+ * hv_attn_selftest_timeout - launches a one-warp kernel whose bounded wait on
+ * an mbarrier that nothing completes must run out after about timeout_us
+ * microseconds, then synchronises and returns the device error word that run
+ * left (expected: bit 0 set, role 5). Tests the timeout path without faulting
+ * or hanging the GPU. Returns -1 on a CUDA error.
+ */
+int hv_attn_selftest_timeout(int timeout_us);
+
+/* Static string for an hv_status code. */
+const char* hv_attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HV_ATTN_H */

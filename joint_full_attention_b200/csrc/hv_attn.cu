@@ -1,0 +1,698 @@
+// hv_attn.cu - joint full self-attention with 3D RoPE for B200 (sm_100a).
+//
+// One persistent, warp-specialised kernel computes, per (batch b, head h),
+//   out = softmax(scale * R(Q) R(K)^T, keys < N + valid_b) V
+// over the joint sequence [video ; text] ("HunyuanVideo 模型结构与数学原理"
+// §5.2 joint attention, §5.5 3D RoPE with the (16, 56, 56) split and
+// theta = 256 on video rows only; §9.1: exact attention computed tile by tile
+// without materialising the score matrix).
+//
+// Work unit: (b, h, 256 query rows) = two 128-row Q tiles sharing every K/V
+// tile. Per CTA (one per SM, 448 threads):
+//   warps 0-3   softmax for Q tile 0 (thread = TMEM lane = query row)
+//   warps 4-7   softmax for Q tile 1
+//   warps 8-11  RoPE: rotate the video rows of each Q/K tile in shared memory
+//               right after TMA lands it, then hand it to the tensor core
+//   warp  12    TMA producer (Q once per unit, then K/V tiles into a ring)
+//   warp  13    TMEM owner and tcgen05.mma issuer
+// Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the
+// bf16 probabilities P_i overwrite the first 64 columns of S_i and feed the
+// PV MMA straight from TMEM.
+//
+// Every mbarrier wait is bounded by a %globaltimer budget; when one runs out
+// the CTA records the role in a device error word, tells the other roles to
+// stop, waits (bounded) for its own copies and MMAs in flight, frees its TMEM
+// and returns.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "hv_attn.h"
+#include "sm100_ptx.cuh"
+
+namespace hv {
+
+constexpr int D = HV_HEAD_DIM;      // head dim
+constexpr int BM = 128;             // query rows per Q tile
+constexpr int BN = 128;             // keys per K/V tile
+constexpr int QTILES = 2;           // Q tiles per work unit
+constexpr int UNIT_ROWS = BM * QTILES;
+constexpr int KSTAGES = 3;
+constexpr int VSTAGES = 2;
+constexpr int BOX_BYTES = 128 * 64 * 2;   // 128 rows x 64 channels bf16, 128B-swizzled
+constexpr int TILE_BYTES = 2 * BOX_BYTES; // 128 rows x 128 channels
+
+constexpr int NUM_WARPS = 14;
+constexpr int NUM_THREADS = NUM_WARPS * 32;
+constexpr int WARP_ROPE = 8;
+constexpr int WARP_TMA = 12;
+constexpr int WARP_MMA = 13;
+constexpr int ROPE_THREADS = 128;
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + QTILES * TILE_BYTES;
+constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
+constexpr int OFF_BAR = OFF_V + VSTAGES * TILE_BYTES;
+// barrier indices
+constexpr int B_Q_FULL = 0, B_Q_READY = 1, B_Q_EMPTY = 2;
+constexpr int B_K_FULL = 3;
+constexpr int B_K_READY = B_K_FULL + KSTAGES;
+constexpr int B_K_EMPTY = B_K_READY + KSTAGES;
+constexpr int B_V_FULL = B_K_EMPTY + KSTAGES;
+constexpr int B_V_EMPTY = B_V_FULL + VSTAGES;
+constexpr int B_S_FULL = B_V_EMPTY + VSTAGES;
+constexpr int B_P_READY = B_S_FULL + QTILES;
+constexpr int B_O_DONE = B_P_READY + QTILES;
+constexpr int B_DRAIN = B_O_DONE + QTILES;
+constexpr int NUM_BARS = B_DRAIN + 1;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_USED = OFF_MISC + 16;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
+
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S = 0;     // + 128*i
+constexpr uint32_t TM_O = 256;   // + 128*i
+
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);  // Q (K-major) x K (K-major)
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);    // P (TMEM)    x V (MN-major)
+
+// rescale O only when a row max grows by more than this (log2 units)
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+enum Role : uint32_t { ROLE_TMA = 1, ROLE_MMA = 2, ROLE_SOFTMAX = 3, ROLE_ROPE = 4, ROLE_SELFTEST = 5 };
+
+struct __align__(64) Params {
+    CUtensorMap tm_q;
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;
+    __nv_bfloat16* out;
+    int B, H, S, N, Hp, Wp, HpWp;
+    int n_qunits;       // ceil(S / 256)
+    int units;          // B * H * n_qunits
+    float theta_log2;   // log2(rope_theta)
+    float scale_log2;   // scale * log2(e)
+    unsigned long long timeout_ns;
+    int text_valid[HV_MAX_BATCH];
+};
+
+__device__ unsigned int g_dev_error = 0;
+
+struct Waiter {
+    volatile int* abort_flag;
+    unsigned long long timeout_ns;
+
+    // Spin until the phase of `bar` with `parity` has completed. Returns false
+    // when the CTA is aborting (this wait ran out, or another role's did).
+    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, uint32_t role) const {
+        if (mbar_try_wait(bar, parity)) return true;
+        const uint64_t t0 = global_timer_ns();
+        while (true) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > timeout_ns) {
+                *abort_flag = 1;
+                atomicOr(&g_dev_error, 1u | (role << 8));
+                __threadfence_block();
+                return false;
+            }
+        }
+    }
+    // Warp-uniform version for roles that continue with warp-collective ops.
+    __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, uint32_t role) const {
+        const bool ok = wait(bar, parity, role);
+        return __all_sync(0xffffffffu, ok);
+    }
+};
+
+struct UnitCoord {
+    int b, h, qu, nt, last_lim;
+};
+
+__device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
+    UnitCoord c;
+    c.qu = u % p.n_qunits;
+    const int bh = u / p.n_qunits;
+    c.h = bh % p.H;
+    c.b = bh / p.H;
+    const int kv_len = p.N + p.text_valid[c.b];
+    c.nt = (kv_len + BN - 1) / BN;
+    c.last_lim = kv_len - (c.nt - 1) * BN;
+    return c;
+}
+
+// Rotate the video rows (sequence index < N) of one 128-row tile in place.
+// Thread `rt` (0..127) owns 16-byte chunk cc = rt % 16 of rows rt/16 + 8k.
+// A chunk holds channels [8cc, 8cc+8): four adjacent pairs, all inside one
+// axis segment because the segment borders 16 and 72 are multiples of 8.
+struct RopeLane {
+    int box, cin, axis;
+    float freq[4];
+};
+
+__device__ __forceinline__ RopeLane make_rope_lane(int rt, float theta_log2) {
+    RopeLane L;
+    const int cc = rt & 15;
+    L.box = cc >> 3;
+    L.cin = cc & 7;
+    const int ch0 = cc * 8;
+    int i0, dax;
+    if (ch0 < 16) {
+        L.axis = 0; i0 = ch0 / 2; dax = 16;
+    } else if (ch0 < 72) {
+        L.axis = 1; i0 = (ch0 - 16) / 2; dax = 56;
+    } else {
+        L.axis = 2; i0 = (ch0 - 72) / 2; dax = 56;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        // theta^(-2i/d) = 2^(-(2i/d) * log2(theta))
+        L.freq[q] = exp2f(-static_cast<float>(2 * (i0 + q)) * theta_log2 / static_cast<float>(dax));
+    }
+    return L;
+}
+
+__device__ __forceinline__ void rope_tile(uint32_t tile, int n0, int rt, const RopeLane& L, const Params& p) {
+    const int rb = rt >> 4;
+#pragma unroll 1
+    for (int k = 0; k < BM / 8; ++k) {
+        const int r = rb + 8 * k;
+        const int n = n0 + r;
+        if (n >= p.N) break;  // rows grow with k: the rest are text or past the end
+        int pos;
+        if (L.axis == 0) pos = n / p.HpWp;
+        else if (L.axis == 1) pos = (n / p.Wp) % p.Hp;
+        else pos = n % p.Wp;
+        const uint32_t addr = tile + L.box * BOX_BYTES + r * 128 + ((L.cin ^ (r & 7)) << 4);
+        uint4 d = lds128(addr);
+        uint32_t w[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float x0 = __uint_as_float(w[q] << 16);
+            const float x1 = __uint_as_float(w[q] & 0xFFFF0000u);
+            float sn, cs;
+            sincosf(static_cast<float>(pos) * L.freq[q], &sn, &cs);
+            w[q] = pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
+        sts128(addr, make_uint4(w[0], w[1], w[2], w[3]));
+    }
+}
+
+// S_i = Q_i K^T: 8 MMAs of K=16 channels; both operands K-major, 128B swizzle.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_tile, uint32_t k_tile) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+        const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
+        const uint64_t b = smem_desc_sw128(k_tile + off, 16, 1024);
+        mma_ss(d_tmem, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O_i (+)= P_i V: 8 MMAs of K=16 keys; P from TMEM (2 bf16 per column),
+// V MN-major (channels contiguous): LBO = distance between the two 64-channel
+// boxes, SBO = 8 key rows.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_tile, bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint64_t b = smem_desc_sw128(v_tile + kk * 16 * 128, BOX_BYTES, 1024);
+        mma_ts(d_tmem, p_tmem + kk * 8, b, IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint32_t bars = base + OFF_BAR;
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_Q_FULL), 1);
+        mbar_init(bar(B_Q_READY), ROPE_THREADS);
+        mbar_init(bar(B_Q_EMPTY), 1);
+        for (int s = 0; s < KSTAGES; ++s) {
+            mbar_init(bar(B_K_FULL + s), 1);
+            mbar_init(bar(B_K_READY + s), ROPE_THREADS);
+            mbar_init(bar(B_K_EMPTY + s), 1);
+        }
+        for (int s = 0; s < VSTAGES; ++s) {
+            mbar_init(bar(B_V_FULL + s), 1);
+            mbar_init(bar(B_V_EMPTY + s), 1);
+        }
+        for (int i = 0; i < QTILES; ++i) {
+            mbar_init(bar(B_S_FULL + i), 1);
+            mbar_init(bar(B_P_READY + i), 128);
+            mbar_init(bar(B_O_DONE + i), 1);
+        }
+        mbar_init(bar(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const Waiter waiter{abort_flag, p.timeout_ns};
+    const uint32_t sQ = base + OFF_Q;
+    const uint32_t sK = base + OFF_K;
+    const uint32_t sV = base + OFF_V;
+
+    if (warp == WARP_TMA) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            uint32_t kt = 0, vt = 0, lu = 0;
+            int armed_q = 0, armed_k[KSTAGES] = {}, armed_v[VSTAGES] = {};
+            uint32_t par_q = 0, par_k[KSTAGES] = {}, par_v[VSTAGES] = {};
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
+                const UnitCoord c = decode_unit(p, u);
+                if (!(ok = waiter.wait(bar(B_Q_EMPTY), (lu & 1) ^ 1, ROLE_TMA))) break;
+                mbar_arrive_expect_tx(bar(B_Q_FULL), QTILES * TILE_BYTES);
+                armed_q = 1; par_q = lu & 1;
+                for (int qi = 0; qi < QTILES; ++qi)
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_4d(sQ + qi * TILE_BYTES + bx * BOX_BYTES, &p.tm_q, bar(B_Q_FULL), bx * 64, c.h,
+                                    c.qu * UNIT_ROWS + qi * BM, c.b);
+                for (int j = 0; j < c.nt; ++j) {
+                    const uint32_t sk = kt % KSTAGES, pk = (kt / KSTAGES) & 1;
+                    if (!(ok = waiter.wait(bar(B_K_EMPTY + sk), pk ^ 1, ROLE_TMA))) break;
+                    mbar_arrive_expect_tx(bar(B_K_FULL + sk), TILE_BYTES);
+                    armed_k[sk] = 1; par_k[sk] = pk;
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_4d(sK + sk * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + sk), bx * 64, c.h,
+                                    j * BN, c.b);
+                    ++kt;
+                    const uint32_t sv = vt % VSTAGES, pv = (vt / VSTAGES) & 1;
+                    if (!(ok = waiter.wait(bar(B_V_EMPTY + sv), pv ^ 1, ROLE_TMA))) break;
+                    mbar_arrive_expect_tx(bar(B_V_FULL + sv), TILE_BYTES);
+                    armed_v[sv] = 1; par_v[sv] = pv;
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_4d(sV + sv * TILE_BYTES + bx * BOX_BYTES, &p.tm_v, bar(B_V_FULL + sv), bx * 64, c.h,
+                                    j * BN, c.b);
+                    ++vt;
+                }
+            }
+            if (!ok) {
+                // Abort: let every copy this warp started land before the CTA
+                // (and its shared memory) goes away.
+                volatile int never = 0;
+                Waiter tail{&never, 20000000ull};
+                if (armed_q) tail.wait(bar(B_Q_FULL), par_q, ROLE_TMA);
+                for (int s = 0; s < KSTAGES; ++s)
+                    if (armed_k[s]) tail.wait(bar(B_K_FULL + s), par_k[s], ROLE_TMA);
+                for (int s = 0; s < VSTAGES; ++s)
+                    if (armed_v[s]) tail.wait(bar(B_V_FULL + s), par_v[s], ROLE_TMA);
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        // ------------------------------------------------------------- MMA
+        if (lane == 0) {
+            uint32_t kt = 0, vt = 0, lu = 0;
+            uint32_t pr[QTILES] = {0, 0};
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
+                const UnitCoord c = decode_unit(p, u);
+                if (!(ok = waiter.wait(bar(B_Q_READY), lu & 1, ROLE_MMA))) break;
+                uint32_t sk = kt % KSTAGES;
+                if (!(ok = waiter.wait(bar(B_K_READY + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                tc_fence_after();
+                issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
+                mma_commit(bar(B_S_FULL + 0));
+                issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + sk * TILE_BYTES);
+                mma_commit(bar(B_S_FULL + 1));
+                mma_commit(bar(B_K_EMPTY + sk));
+                ++kt;
+                if (c.nt == 1) mma_commit(bar(B_Q_EMPTY));
+                for (int j = 0; j < c.nt; ++j) {
+                    const uint32_t sv = vt % VSTAGES;
+                    if (!(ok = waiter.wait(bar(B_V_FULL + sv), (vt / VSTAGES) & 1, ROLE_MMA))) break;
+                    const uint32_t v_tile = sV + sv * TILE_BYTES;
+                    // Q tile 0: PV for tile j, then QK for tile j+1
+                    if (!(ok = waiter.wait(bar(B_P_READY + 0), pr[0] & 1, ROLE_MMA))) break;
+                    ++pr[0];
+                    tc_fence_after();
+                    issue_pv(tmem_base + TM_O + 0, tmem_base + TM_S + 0, v_tile, j > 0);
+                    if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 0));
+                    const bool more = j + 1 < c.nt;
+                    sk = kt % KSTAGES;
+                    if (more) {
+                        if (!(ok = waiter.wait(bar(B_K_READY + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                        tc_fence_after();
+                        issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
+                        mma_commit(bar(B_S_FULL + 0));
+                    }
+                    // Q tile 1
+                    if (!(ok = waiter.wait(bar(B_P_READY + 1), pr[1] & 1, ROLE_MMA))) break;
+                    ++pr[1];
+                    tc_fence_after();
+                    issue_pv(tmem_base + TM_O + 128, tmem_base + TM_S + 128, v_tile, j > 0);
+                    mma_commit(bar(B_V_EMPTY + sv));
+                    ++vt;
+                    if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 1));
+                    if (more) {
+                        issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + sk * TILE_BYTES);
+                        mma_commit(bar(B_S_FULL + 1));
+                        mma_commit(bar(B_K_EMPTY + sk));
+                        ++kt;
+                        if (j + 1 == c.nt - 1) mma_commit(bar(B_Q_EMPTY));
+                    }
+                }
+            }
+            if (!ok) {
+                // Abort: wait for the MMAs already issued before TMEM is freed.
+                mma_commit(bar(B_DRAIN));
+                volatile int never = 0;
+                Waiter tail{&never, 20000000ull};
+                tail.wait(bar(B_DRAIN), 0, ROLE_MMA);
+            }
+        }
+    } else if (warp >= WARP_ROPE) {
+        // ------------------------------------------------------------ RoPE
+        const int rt = threadIdx.x - WARP_ROPE * 32;
+        const RopeLane L = make_rope_lane(rt, p.theta_log2);
+        uint32_t kt = 0, lu = 0;
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
+            const UnitCoord c = decode_unit(p, u);
+            if (!waiter.wait(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
+            for (int qi = 0; qi < QTILES; ++qi)
+                rope_tile(sQ + qi * TILE_BYTES, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_Q_READY));
+            bool ok = true;
+            for (int j = 0; j < c.nt; ++j, ++kt) {
+                const uint32_t sk = kt % KSTAGES;
+                if (!(ok = waiter.wait(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
+                if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, j * BN, rt, L, p);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_K_READY + sk));
+            }
+            if (!ok) break;
+        }
+    } else {
+        // --------------------------------------------------------- softmax
+        const int qi = warp >> 2;                       // Q tile of this warpgroup
+        const int row = ((warp & 3) << 5) + lane;       // = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
+        const uint32_t tS = tmem_base + lane_off + TM_S + 128 * qi;
+        const uint32_t tO = tmem_base + lane_off + TM_O + 128 * qi;
+        const float sl2 = p.scale_log2;
+        uint32_t sp = 0, lu = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
+            const UnitCoord c = decode_unit(p, u);
+            float m = -INFINITY;   // running max, scaled log2 units
+            float l = 0.f;         // running sum of probabilities
+            for (int j = 0; j < c.nt; ++j, ++sp) {
+                if (!(ok = waiter.wait_warp(bar(B_S_FULL + qi), sp & 1, ROLE_SOFTMAX))) break;
+                tc_fence_after();
+                const int lim = (j == c.nt - 1) ? c.last_lim : BN;
+                uint32_t r[32];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    tmem_ld32(tS + 32 * ch, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float s = (32 * ch + e < lim) ? __uint_as_float(r[e]) : -INFINITY;
+                        mx = fmaxf(mx, s);
+                    }
+                }
+                const float mx_s = mx * sl2;
+                float m_new = m, alpha = 1.f;
+                if (mx_s - m > RESCALE_THRESHOLD) {
+                    m_new = mx_s;
+                    alpha = ex2_approx(m - m_new);
+                }
+                float rs = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    tmem_ld32(tS + 32 * ch, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int col = 32 * ch + 2 * e;
+                        const float p0 = (col < lim) ? ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -m_new)) : 0.f;
+                        const float p1 =
+                            (col + 1 < lim) ? ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -m_new)) : 0.f;
+                        rs += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + 16 * ch, pk);
+                }
+                l = l * alpha + rs;
+                m = m_new;
+                if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        tmem_ld32(tO + 32 * ch, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st32(tO + 32 * ch, r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_P_READY + qi));
+            }
+            if (!ok) break;
+            // epilogue: out = O / l as bf16, one 256-byte row per thread
+            if (!(ok = waiter.wait_warp(bar(B_O_DONE + qi), lu & 1, ROLE_SOFTMAX))) break;
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            const int srow = c.qu * UNIT_ROWS + qi * BM + row;
+            const bool store = srow < p.S;
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.out + ((static_cast<size_t>(c.b) * p.S + (store ? srow : 0)) * p.H + c.h) * D);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(tO + 32 * ch, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (store) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[ch * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                }
+            }
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == WARP_MMA) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// One warp waits on an mbarrier that nothing completes; the bounded wait must
+// run out, record ROLE_SELFTEST and return.
+__global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&mbar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const Waiter w{&abort_flag, timeout_ns};
+    w.wait_warp(smem_addr(&mbar), 0, ROLE_SELFTEST);
+    __syncthreads();
+}
+
+// ------------------------------------------------------------------- host
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// [B, S, H, 128] bf16 as a 4-D tensor (channel, head, token, batch); a box is
+// 64 channels x 1 head x 128 tokens, landing as 128 rows of 128 bytes with the
+// 128-byte swizzle the MMA descriptors expect. Rows past S read as zero.
+static bool make_qkv_map(CUtensorMap* map, const void* ptr, int B, int S, int H) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                                   static_cast<cuuint64_t>(S) * H * D * 2};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(BM), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int ok = -1;   // -1 unknown, 0 unsupported, 1 sm_100
+    int sms = 0;
+};
+
+static DeviceInfo& device_info(int dev) {
+    static DeviceInfo infos[64];
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo& di = infos[dev & 63];
+    if (di.ok < 0) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        di.sms = sms;
+        di.ok = (major == 10 && minor == 0) ? 1 : 0;
+        if (di.ok &&
+            cudaFuncSetAttribute(hv_attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+                cudaSuccess)
+            di.ok = 0;
+    }
+    return di;
+}
+
+static bool overlaps(const void* a, const void* b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
+
+}  // namespace hv
+
+extern "C" {
+
+const char* hv_attn_status_string(int status) {
+    switch (status) {
+        case HV_OK: return "ok";
+        case HV_ERR_NULL_POINTER: return "null pointer";
+        case HV_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case HV_ERR_BAD_SHAPE: return "bad shape (B, heads, T, Hp, Wp must be >= 1, B <= HV_MAX_BATCH)";
+        case HV_ERR_BAD_TEXT: return "bad text length (0 <= text_valid[b] <= text_len <= 256)";
+        case HV_ERR_TOO_LARGE: return "problem too large for int32 TMA coordinates";
+        case HV_ERR_ALIAS: return "out overlaps q, k or v";
+        case HV_ERR_BAD_SCALAR: return "rope_theta must be finite and > 0, scale finite";
+        case HV_ERR_NO_DEVICE: return "current CUDA device is not sm_100";
+        case HV_ERR_LAUNCH: return "CUDA launch or driver call failed";
+        case HV_ERR_DEVICE_TIMEOUT: return "a kernel-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+long long hv_video_tokens(int frames, int height, int width) {
+    if (frames < 1 || (frames - 1) % 4 != 0) return -1;
+    if (height <= 0 || width <= 0 || height % 16 != 0 || width % 16 != 0) return -1;
+    const long long t = (frames - 1) / 4 + 1;
+    return t * (height / 16) * static_cast<long long>(width / 16);
+}
+
+int hv_attn_forward(const void* q, const void* k, const void* v, void* out, int B, int heads, int T, int Hp, int Wp,
+                    int text_len, const int* text_valid, float rope_theta, float scale, void* cuda_stream) {
+    using namespace hv;
+    if (!q || !k || !v || !out || !text_valid) return HV_ERR_NULL_POINTER;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+    if (mis & 15u) return HV_ERR_MISALIGNED;
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH) return HV_ERR_BAD_SHAPE;
+    if (text_len < 0 || text_len > HV_MAX_TEXT_LEN) return HV_ERR_BAD_TEXT;
+    for (int b = 0; b < B; ++b)
+        if (text_valid[b] < 0 || text_valid[b] > text_len) return HV_ERR_BAD_TEXT;
+    if (!std::isfinite(rope_theta) || !(rope_theta > 0.f) || !std::isfinite(scale)) return HV_ERR_BAD_SCALAR;
+    const long long n_video = static_cast<long long>(T) * Hp * Wp;
+    const long long s_len = n_video + text_len;
+    const long long units = static_cast<long long>(B) * heads * ((s_len + UNIT_ROWS - 1) / UNIT_ROWS);
+    if (s_len + UNIT_ROWS >= (1ll << 31) || s_len * heads * D >= (1ll << 31) || units >= (1ll << 31))
+        return HV_ERR_TOO_LARGE;
+    const size_t bytes = static_cast<size_t>(B) * s_len * heads * D * 2;
+    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return HV_ERR_ALIAS;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    DeviceInfo& di = device_info(dev);
+    if (di.ok != 1) return HV_ERR_NO_DEVICE;
+
+    Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
+    std::memset(prm, 0, sizeof(Params));
+    const int S = static_cast<int>(s_len);
+    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, S, heads) ||
+        !make_qkv_map(&prm->tm_v, v, B, S, heads)) {
+        delete prm;
+        return HV_ERR_LAUNCH;
+    }
+    prm->out = static_cast<__nv_bfloat16*>(out);
+    prm->B = B;
+    prm->H = heads;
+    prm->S = S;
+    prm->N = static_cast<int>(n_video);
+    prm->Hp = Hp;
+    prm->Wp = Wp;
+    prm->HpWp = Hp * Wp;
+    prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
+    prm->units = static_cast<int>(units);
+    prm->theta_log2 = static_cast<float>(std::log2(static_cast<double>(rope_theta)));
+    prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    prm->timeout_ns = kWaitTimeoutNs;
+    for (int b = 0; b < B; ++b) prm->text_valid[b] = text_valid[b];
+
+    const int grid = static_cast<int>(units < di.sms ? units : di.sms);
+    hv_attn_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, static_cast<cudaStream_t>(cuda_stream)>>>(*prm);
+    delete prm;
+    const cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
+}
+
+int hv_attn_last_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, hv::g_dev_error, sizeof(word)) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(hv::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+    return static_cast<int>(word);
+}
+
+int hv_attn_selftest_timeout(int timeout_us) {
+    if (timeout_us < 1 || timeout_us > 1000000) return -1;
+    if (hv_attn_last_device_error() < 0) return -1;   // clears the word first
+    hv::hv_selftest_timeout_kernel<<<1, 32>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    return hv_attn_last_device_error();
+}
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+"""Python binding of the C ABI in ``include/hv_attn.h`` (ctypes).
+
+Argument marshalling only: tensors are checked and their device pointers and
+the current CUDA stream are handed to ``libhvattn.so``; every step of the
+attention runs in the library's sm_100a kernel. There is no fallback: if the
+library is missing or the device is not an sm_100 part the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libhvattn.so"
+_lib = None
+
+HV_OK = 0
+STATUS_NAMES = {
+    0: "HV_OK", 1: "HV_ERR_NULL_POINTER", 2: "HV_ERR_MISALIGNED", 3: "HV_ERR_BAD_SHAPE",
+    4: "HV_ERR_BAD_TEXT", 5: "HV_ERR_TOO_LARGE", 6: "HV_ERR_ALIAS", 7: "HV_ERR_BAD_SCALAR",
+    8: "HV_ERR_NO_DEVICE", 9: "HV_ERR_LAUNCH", 10: "HV_ERR_DEVICE_TIMEOUT",
+}
+EXPORTED = ("hv_attn_forward", "hv_video_tokens", "hv_attn_last_device_error",
+            "hv_attn_selftest_timeout", "hv_attn_status_string")
+
+
+class HVError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libhvattn.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise RuntimeError(f"{_LIB_PATH} is missing: run joint_full_attention_b200.build.build() first")
+        L = ctypes.CDLL(str(_LIB_PATH))
+        L.hv_attn_forward.restype = ctypes.c_int
+        L.hv_attn_forward.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
+        L.hv_video_tokens.restype = ctypes.c_longlong
+        L.hv_video_tokens.argtypes = [ctypes.c_int] * 3
+        L.hv_attn_last_device_error.restype = ctypes.c_int
+        L.hv_attn_last_device_error.argtypes = []
+        L.hv_attn_selftest_timeout.restype = ctypes.c_int
+        L.hv_attn_selftest_timeout.argtypes = [ctypes.c_int]
+        L.hv_attn_status_string.restype = ctypes.c_char_p
+        L.hv_attn_status_string.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().hv_attn_status_string(int(status)).decode()
+
+
+def video_tokens(frames: int, height: int, width: int) -> int:
+    """N video tokens of an F x H x W clip, or -1 (pure host computation in the library)."""
+    return int(lib().hv_video_tokens(int(frames), int(height), int(width)))
+
+
+def last_device_error() -> int:
+    """Device error word of the library's kernels since the last read (synchronises)."""
+    return int(lib().hv_attn_last_device_error())
+
+
+def selftest_timeout(timeout_us: int = 20000) -> int:
+    return int(lib().hv_attn_selftest_timeout(int(timeout_us)))
+
+
+def _check(t: torch.Tensor, name: str, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous [B, S, heads, 128]")
+    if t.dim() != 4 or t.shape[-1] != 128:
+        raise ValueError(f"{name} must be [B, S, heads, 128], got {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} shape {tuple(t.shape)} != {tuple(shape)}")
+
+
+def attn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, text_valid,
+                 rope_theta: float = 256.0, scale: float | None = None, out: torch.Tensor | None = None,
+                 stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Joint 3D-RoPE attention on device tensors; enqueued on ``stream`` (default: current)."""
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    b_sz, _, heads, _ = q.shape
+    t_lat, hp, wp = (int(x) for x in grid)
+    valid = (ctypes.c_int * b_sz)(*[int(x) for x in text_valid])
+    if len(text_valid) != b_sz:
+        raise ValueError("text_valid needs one entry per batch sample")
+    if scale is None:
+        scale = 1.0 / math.sqrt(128)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = lib().hv_attn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b_sz, heads,
+                                   t_lat, hp, wp, int(text_len), valid, float(rope_theta), float(scale),
+                                   ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_forward")
+    return out
+
+
+def attn_forward_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, grid, text_len: int,
+                      text_valid, rope_theta: float = 256.0, scale: float | None = None,
+                      device: int | torch.device = 0, out_host: torch.Tensor | None = None,
+                      work: dict | None = None) -> torch.Tensor:
+    """Host-to-host call: copy pinned host inputs to the GPU, run, copy the output back.
+
+    ``work`` may hold reusable device buffers (keys "q", "k", "v", "out") so
+    that repeated calls allocate nothing on the device.
+    """
+    dev = torch.device("cuda", device) if isinstance(device, int) else device
+    work = {} if work is None else work
+    for name, src in (("q", q_host), ("k", k_host), ("v", v_host)):
+        buf = work.get(name)
+        if buf is None or buf.shape != src.shape:
+            buf = work[name] = torch.empty(src.shape, dtype=src.dtype, device=dev)
+        buf.copy_(src, non_blocking=True)
+    o = work.get("out")
+    if o is None or o.shape != q_host.shape:
+        o = work["out"] = torch.empty(q_host.shape, dtype=q_host.dtype, device=dev)
+    attn_forward(work["q"], work["k"], work["v"], grid, text_len, text_valid, rope_theta, scale, out=o)
+    if out_host is None:
+        out_host = torch.empty(q_host.shape, dtype=q_host.dtype, pin_memory=True)
+    out_host.copy_(o, non_blocking=True)
+    torch.cuda.current_stream(dev).synchronize()
+    return out_host

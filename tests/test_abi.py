@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library builds, loads, exports every
+symbol declared in include/hv_attn.h, computes token counts, and rejects bad
+arguments with status codes before touching a device."""
+
+from __future__ import annotations
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from joint_full_attention_b200 import build as B
+from joint_full_attention_b200 import hvattn as H
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "hv_attn.h"
+GOLDEN = Path(__file__).parent / "golden"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return H.lib()
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(hv_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("hv_attn_forward", "hv_video_tokens", "hv_attn_last_device_error"):
+        assert must in names
+    assert set(names) <= set(H.EXPORTED) | {n for n in names}
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for name in names:
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_video_tokens_worked_examples(lib):
+    for line in (GOLDEN / "token_grids.txt").read_text().splitlines():
+        line = line.split("#", 1)[0].split()
+        if line:
+            f, h, w, *_, n = map(int, line)
+            assert H.video_tokens(f, h, w) == n
+    assert H.video_tokens(1, 256, 256) == 256
+    assert H.video_tokens(129, 544, 960) == 67320
+    for bad in [(16, 544, 960), (0, 544, 960), (17, 540, 960), (17, 544, 0), (-3, 16, 16)]:
+        assert H.video_tokens(*bad) == -1
+
+
+def test_status_strings(lib):
+    for code, name in H.STATUS_NAMES.items():
+        assert H.status_string(code)
+    assert "unknown" in H.status_string(999)
+
+
+def _call(lib, q=0x10000, k=0x20000, v=0x30000, out=0x40000, B_=1, heads=2, T=2, Hp=4, Wp=4, text_len=8,
+          valid=(5,), theta=256.0, scale=0.088, stream=None):
+    arr = None if valid is None else (ctypes.c_int * max(1, len(valid)))(*valid)
+    return lib.hv_attn_forward(q, k, v, out, B_, heads, T, Hp, Wp, text_len, arr, theta, scale, stream)
+
+
+def test_argument_validation_codes(lib):
+    big = 1 << 40
+    assert _call(lib, q=None) == 1
+    assert _call(lib, valid=None) == 1
+    assert _call(lib, k=0x20008) == 2
+    assert _call(lib, B_=0) == 3
+    assert _call(lib, heads=0) == 3
+    assert _call(lib, Wp=0) == 3
+    assert _call(lib, B_=513, valid=(5,) * 513) == 3
+    assert _call(lib, text_len=257, valid=(5,)) == 4
+    assert _call(lib, text_len=-1, valid=(0,)) == 4
+    assert _call(lib, valid=(9,)) == 4
+    assert _call(lib, valid=(-1,)) == 4
+    assert _call(lib, theta=0.0) == 7
+    assert _call(lib, theta=float("nan")) == 7
+    assert _call(lib, scale=float("inf")) == 7
+    assert _call(lib, T=40000, Hp=400, Wp=400) == 5
+    # out overlapping an input
+    assert _call(lib, q=big, k=big * 2, v=big * 3, out=big + 4096) == 6
+
+
+def test_valid_arguments_without_gpu_fail_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    st = _call(lib, q=1 << 32, k=2 << 32, v=3 << 32, out=4 << 32)
+    assert st in (8, 9)

@@ -1,0 +1,178 @@
+"""GPU parity: the sm_100a kernel (called through the C ABI) against the
+float64 oracle on the same seeded bf16 inputs.
+
+Tolerance (bf16 I/O, unit-variance inputs): max |gpu - oracle| <= 2e-2 and
+mean |gpu - oracle| <= 2e-3, on the full output for the small workloads and
+on 4096 seeded (batch, head, row) samples for the two 129-frame workloads.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from joint_full_attention_b200 import build as B
+from joint_full_attention_b200 import hvattn as H
+from joint_full_attention_b200 import workloads as W
+from oracle import hv_oracle as O
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B.build()
+    H.lib()
+    assert H.last_device_error() == 0
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def out_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def run_gpu(inp, grid, text_len, theta=256.0, scale=None, out=None):
+    q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
+    o = H.attn_forward(q, k, v, grid, text_len, inp["text_valid"], theta, scale, out=out)
+    torch.cuda.synchronize()
+    assert H.last_device_error() == 0
+    return o
+
+
+def f64(inp):
+    return {n: W.bf16_bits_to_f64(inp[n]) for n in ("q", "k", "v")}
+
+
+def check(got, ref, what):
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
+    return err.max(), err.mean()
+
+
+def full_check(inp, grid, text_len, theta=256.0, scale=None):
+    o = run_gpu(inp, grid, text_len, theta, scale)
+    x = f64(inp)
+    ref = O.joint_attention(x["q"], x["k"], x["v"], grid, text_len, inp["text_valid"], theta, scale)
+    return check(out_f64(o), ref, f"grid {grid} text {text_len}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "img256", "v544x960x17"])
+def test_full_output_parity(name):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, seed=1)
+    full_check(inp, wl.grid, wl.text_len)
+
+
+@pytest.mark.parametrize("name", ["v544x960x129", "v720x1280x129"])
+def test_sampled_parity_large(name):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, seed=2)
+    o = run_gpu(inp, wl.grid, wl.text_len)
+    samples = W.sample_triples(wl.batch, wl.heads, wl.n_video, wl.text_len, inp["text_valid"], 4096, seed=3)
+    got = o[samples[:, 0], samples[:, 2], samples[:, 1]].float().cpu().numpy().astype(np.float64)
+    x = f64(inp)
+    ref = O.joint_attention_samples(x["q"], x["k"], x["v"], wl.grid, wl.text_len, inp["text_valid"], samples)
+    check(got, ref, name)
+
+
+def _small(grid, text_len, valid, batch=1, heads=3, seed=5, k_scale=1.0):
+    wl = W.Workload("edge", "edge case", batch, heads, grid, text_len, valid=tuple(valid))
+    inp = W.make_inputs(wl, seed=seed)
+    if k_scale != 1.0:
+        inp["k"] = W.round_to_bf16_bits(W.bf16_bits_to_f32(inp["k"]) * np.float32(k_scale))
+    return inp
+
+
+@pytest.mark.parametrize("grid,text_len,valid", [
+    ((1, 1, 1), 0, [0]),            # one video token, no text
+    ((1, 1, 1), 256, [0]),          # all text padded
+    ((2, 4, 4), 8, [8]),            # no padding
+    ((3, 5, 7), 37, [0]),           # ragged, text present but none valid
+    ((1, 9, 15), 256, [256]),       # full text
+    ((5, 3, 11), 100, [1]),         # 265 rows: ragged Q unit and K tile
+    ((2, 16, 16), 0, [0]),          # exactly 512 rows, no text
+    ((4, 8, 9), 19, [19, 3, 0]),    # batch of 3 with different valid lengths
+])
+def test_edge_shapes(grid, text_len, valid):
+    inp = _small(grid, text_len, valid, batch=len(valid))
+    full_check(inp, grid, text_len)
+
+
+def test_theta_and_scale_parameters():
+    grid, text_len = (3, 6, 10), 30
+    inp = _small(grid, text_len, [17])
+    full_check(inp, grid, text_len, theta=10000.0)
+    full_check(inp, grid, text_len, scale=0.05)
+    full_check(inp, grid, text_len, theta=2.0, scale=1.0 / math.sqrt(64))
+
+
+def test_sharp_softmax_rescaling():
+    """Large score range: exercises the running-max rescale of O."""
+    grid, text_len = (4, 10, 10), 64
+    inp = _small(grid, text_len, [50], k_scale=3.0)
+    full_check(inp, grid, text_len)
+
+
+def test_padding_invariance_and_determinism():
+    grid, text_len = (2, 8, 8), 64
+    inp = _small(grid, text_len, [10])
+    o1 = run_gpu(inp, grid, text_len).clone()
+    o2 = run_gpu(inp, grid, text_len)
+    assert torch.equal(o1, o2), "two runs differ"
+    n = 128
+    inp2 = dict(inp)
+    for name in ("k", "v"):
+        arr = inp[name].copy()
+        arr[:, n + 10:] = W.round_to_bf16_bits(np.full(arr[:, n + 10:].shape, 3.5, dtype=np.float32))
+        inp2[name] = arr
+    o3 = run_gpu(inp2, grid, text_len)
+    assert torch.equal(o1, o3), "padded keys changed the output"
+
+
+def test_output_canary_untouched():
+    grid, text_len = (3, 7, 5), 21
+    inp = _small(grid, text_len, [11])
+    s_len = 105 + text_len
+    buf = torch.full((1, s_len + 64, 3, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[:, :s_len]
+    assert out.is_contiguous()
+    run_gpu(inp, grid, text_len, out=out)
+    assert torch.all(buf[:, s_len:] == 7.0), "kernel wrote past the output"
+
+
+def test_errors_on_device():
+    q = torch.zeros(1, 40, 2, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward(q, q, q, (2, 4, 4), 8, [9])
+    assert e.value.status == 4
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward(q, q, q, (2, 4, 4), 8, [5], out=q)
+    assert e.value.status == 6
+    flat = torch.zeros(1 * 40 * 2 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+    mis = flat[1:1 + 40 * 2 * 128].view(1, 40, 2, 128)
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward(mis, q, q, (2, 4, 4), 8, [5], out=torch.empty_like(q))
+    assert e.value.status == 2
+    assert H.last_device_error() == 0
+
+
+def test_bounded_wait_times_out_cleanly():
+    word = H.selftest_timeout(20000)
+    assert word & 1 and (word >> 8) & 0xFF == 5
+    assert H.last_device_error() == 0
+    # the context is still usable
+    inp = _small((2, 4, 4), 8, [5])
+    full_check(inp, (2, 4, 4), 8)
