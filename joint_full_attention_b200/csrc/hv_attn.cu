@@ -8,13 +8,16 @@
 // without materialising the score matrix).
 //
 // Work unit: (b, h, 256 query rows) = two 128-row Q tiles sharing every K/V
-// tile. Per CTA (one per SM, 448 threads):
+// tile. Per CTA (one per SM, 512 threads = 4 warpgroups):
 //   warps 0-3   softmax for Q tile 0 (thread = TMEM lane = query row)
 //   warps 4-7   softmax for Q tile 1
 //   warps 8-11  RoPE: rotate the video rows of each Q/K tile in shared memory
 //               right after TMA lands it, then hand it to the tensor core
 //   warp  12    TMA producer (Q once per unit, then K/V tiles into a ring)
 //   warp  13    TMEM owner and tcgen05.mma issuer
+//   warps 14-15 idle (complete the last warpgroup)
+// setmaxnreg moves registers to the softmax warpgroups, which hold a full
+// 128-column score row per thread.
 // Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the
 // bf16 probabilities P_i overwrite the first 64 columns of S_i and feed the
 // PV MMA straight from TMEM.
@@ -44,23 +47,34 @@ constexpr int BM = 128;             // query rows per Q tile
 constexpr int BN = 128;             // keys per K/V tile
 constexpr int QTILES = 2;           // Q tiles per work unit
 constexpr int UNIT_ROWS = BM * QTILES;
-constexpr int KSTAGES = 3;
+constexpr int KSTAGES = 2;
 constexpr int VSTAGES = 2;
 constexpr int BOX_BYTES = 128 * 64 * 2;   // 128 rows x 64 channels bf16, 128B-swizzled
 constexpr int TILE_BYTES = 2 * BOX_BYTES; // 128 rows x 128 channels
 
-constexpr int NUM_WARPS = 14;
+constexpr int NUM_WARPS = 16;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
 constexpr int WARP_ROPE = 8;
 constexpr int WARP_TMA = 12;
 constexpr int WARP_MMA = 13;
 constexpr int ROPE_THREADS = 128;
+// per-thread registers after setmaxnreg: 2 x 128 x 176 + 128 x 64 + 128 x 96
+// = 65536 = 512 threads x 128 registers at launch
+constexpr uint32_t REGS_SOFTMAX = 176;
+constexpr uint32_t REGS_ROPE = 64;
+constexpr uint32_t REGS_CONTROL = 96;
+static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL <= NUM_WARPS * 32 * 128,
+              "register split exceeds the launch allocation");
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + QTILES * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
-constexpr int OFF_BAR = OFF_V + VSTAGES * TILE_BYTES;
+// cos/sin table of the rotation angles: float2 (cos, sin) per (axis, position,
+// pair) = 8*T + 28*(Hp + Wp) entries, built once per CTA.
+constexpr int OFF_TABLE = OFF_V + VSTAGES * TILE_BYTES;
+constexpr int TABLE_MAX_ENTRIES = 4096;
+constexpr int OFF_BAR = OFF_TABLE + TABLE_MAX_ENTRIES * 8;
 // barrier indices
 constexpr int B_Q_FULL = 0, B_Q_READY = 1, B_Q_EMPTY = 2;
 constexpr int B_K_FULL = 3;
@@ -95,7 +109,8 @@ struct __align__(64) Params {
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     __nv_bfloat16* out;
-    int B, H, S, N, Hp, Wp, HpWp;
+    int B, H, S, N, T, Hp, Wp, HpWp;
+    int use_table;      // 1: cos/sin from the shared-memory table, 0: sincosf per pair
     int n_qunits;       // ceil(S / 256)
     int units;          // B * H * n_qunits
     float theta_log2;   // log2(rope_theta)
@@ -153,56 +168,114 @@ __device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
 // Thread `rt` (0..127) owns 16-byte chunk cc = rt % 16 of rows rt/16 + 8k.
 // A chunk holds channels [8cc, 8cc+8): four adjacent pairs, all inside one
 // axis segment because the segment borders 16 and 72 are multiples of 8.
+// Axis t: channels [0,16), 8 pairs; h: [16,72), 28 pairs; w: [72,128), 28 pairs.
 struct RopeLane {
     int box, cin, axis;
+    int i0;            // first pair index of the chunk inside its axis segment
+    int half_dim;      // pairs in the axis segment (8 or 28)
+    int table_base;    // first table entry of the axis segment
     float freq[4];
 };
 
-__device__ __forceinline__ RopeLane make_rope_lane(int rt, float theta_log2) {
+// Angles are passed to sincospif in units of pi: sin(pi*x) needs no
+// argument reduction beyond taking x modulo 2.
+constexpr float kInvPi = 0.318309886183790672f;
+
+__device__ __forceinline__ float axis_freq(int i, int dax, float theta_log2) {
+    // theta^(-2i/d) = 2^(-(2i/d) * log2(theta))
+    return exp2f(-static_cast<float>(2 * i) * theta_log2 / static_cast<float>(dax));
+}
+
+__device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
     RopeLane L;
     const int cc = rt & 15;
     L.box = cc >> 3;
     L.cin = cc & 7;
     const int ch0 = cc * 8;
-    int i0, dax;
+    int dax;
     if (ch0 < 16) {
-        L.axis = 0; i0 = ch0 / 2; dax = 16;
+        L.axis = 0; L.i0 = ch0 / 2; dax = 16; L.table_base = 0;
     } else if (ch0 < 72) {
-        L.axis = 1; i0 = (ch0 - 16) / 2; dax = 56;
+        L.axis = 1; L.i0 = (ch0 - 16) / 2; dax = 56; L.table_base = 8 * p.T;
     } else {
-        L.axis = 2; i0 = (ch0 - 72) / 2; dax = 56;
+        L.axis = 2; L.i0 = (ch0 - 72) / 2; dax = 56; L.table_base = 8 * p.T + 28 * p.Hp;
     }
+    L.half_dim = dax / 2;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        // theta^(-2i/d) = 2^(-(2i/d) * log2(theta))
-        L.freq[q] = exp2f(-static_cast<float>(2 * (i0 + q)) * theta_log2 / static_cast<float>(dax));
-    }
+    for (int q = 0; q < 4; ++q) L.freq[q] = axis_freq(L.i0 + q, dax, p.theta_log2);
     return L;
 }
 
-__device__ __forceinline__ void rope_tile(uint32_t tile, int n0, int rt, const RopeLane& L, const Params& p) {
+// Fill the (cos, sin) table: entry e of axis a at position pos and pair i
+// holds the rotation by pos * theta^(-2i/d_a).
+__device__ __forceinline__ void build_rope_table(float2* table, const Params& p) {
+    const int n_t = 8 * p.T, n_h = 28 * p.Hp, n_w = 28 * p.Wp;
+    for (int e = threadIdx.x; e < n_t + n_h + n_w; e += blockDim.x) {
+        int pos, i, dax;
+        if (e < n_t) {
+            pos = e / 8; i = e % 8; dax = 16;
+        } else if (e < n_t + n_h) {
+            pos = (e - n_t) / 28; i = (e - n_t) % 28; dax = 56;
+        } else {
+            pos = (e - n_t - n_h) / 28; i = (e - n_t - n_h) % 28; dax = 56;
+        }
+        float sn, cs;
+        sincospif(static_cast<float>(pos) * axis_freq(i, dax, p.theta_log2) * kInvPi, &sn, &cs);
+        table[e] = make_float2(cs, sn);
+    }
+}
+
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
+    const float x0 = __uint_as_float(w << 16);          // channel 2i   (low half)
+    const float x1 = __uint_as_float(w & 0xFFFF0000u);  // channel 2i+1 (high half)
+    return pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+}
+
+__device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int rt, const RopeLane& L,
+                                          const Params& p) {
     const int rb = rt >> 4;
+    int n = n0 + rb;
+    if (n >= p.N) return;
+    // (t, h, w) of row rb, then stepped by 8 rows at a time
+    int w = n % p.Wp;
+    const int th = n / p.Wp;
+    int h = th % p.Hp;
+    int t = th / p.Hp;
 #pragma unroll 1
     for (int k = 0; k < BM / 8; ++k) {
         const int r = rb + 8 * k;
-        const int n = n0 + r;
-        if (n >= p.N) break;  // rows grow with k: the rest are text or past the end
-        int pos;
-        if (L.axis == 0) pos = n / p.HpWp;
-        else if (L.axis == 1) pos = (n / p.Wp) % p.Hp;
-        else pos = n % p.Wp;
+        const int pos = L.axis == 0 ? t : (L.axis == 1 ? h : w);
         const uint32_t addr = tile + L.box * BOX_BYTES + r * 128 + ((L.cin ^ (r & 7)) << 4);
         uint4 d = lds128(addr);
-        uint32_t w[4] = {d.x, d.y, d.z, d.w};
+        if (p.use_table) {
+            const uint32_t ta = table + 8u * static_cast<uint32_t>(L.table_base + pos * L.half_dim + L.i0);
+            const uint4 c01 = lds128(ta);
+            const uint4 c23 = lds128(ta + 16);
+            d.x = rotate_pair(d.x, __uint_as_float(c01.x), __uint_as_float(c01.y));
+            d.y = rotate_pair(d.y, __uint_as_float(c01.z), __uint_as_float(c01.w));
+            d.z = rotate_pair(d.z, __uint_as_float(c23.x), __uint_as_float(c23.y));
+            d.w = rotate_pair(d.w, __uint_as_float(c23.z), __uint_as_float(c23.w));
+        } else {
+            uint32_t wv[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float x0 = __uint_as_float(w[q] << 16);
-            const float x1 = __uint_as_float(w[q] & 0xFFFF0000u);
-            float sn, cs;
-            sincosf(static_cast<float>(pos) * L.freq[q], &sn, &cs);
-            w[q] = pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+            for (int q = 0; q < 4; ++q) {
+                float sn, cs;
+                sincospif(static_cast<float>(pos) * L.freq[q] * kInvPi, &sn, &cs);
+                wv[q] = rotate_pair(wv[q], cs, sn);
+            }
+            d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        sts128(addr, make_uint4(w[0], w[1], w[2], w[3]));
+        sts128(addr, d);
+        n += 8;
+        if (n >= p.N) break;  // rows only grow: the rest are text or past the end
+        w += 8;
+        while (w >= p.Wp) {
+            w -= p.Wp;
+            if (++h == p.Hp) {
+                h = 0;
+                ++t;
+            }
+        }
     }
 }
 
@@ -268,6 +341,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
+    if (p.use_table) build_rope_table(reinterpret_cast<float2*>(base_ptr + OFF_TABLE), p);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -277,16 +351,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     const uint32_t sQ = base + OFF_Q;
     const uint32_t sK = base + OFF_K;
     const uint32_t sV = base + OFF_V;
+    const uint32_t sTable = base + OFF_TABLE;
 
-    if (warp == WARP_TMA) {
+    if (warp >= WARP_TMA) {
+      regs_decrease<REGS_CONTROL>();
+      if (warp == WARP_TMA) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&p.tm_q);
             tma_prefetch_desc(&p.tm_k);
             tma_prefetch_desc(&p.tm_v);
             uint32_t kt = 0, vt = 0, lu = 0;
-            int armed_q = 0, armed_k[KSTAGES] = {}, armed_v[VSTAGES] = {};
-            uint32_t par_q = 0, par_k[KSTAGES] = {}, par_v[VSTAGES] = {};
+            // stages with a load in flight and the parity it completes (bit per stage)
+            uint32_t armed_q = 0, armed_k = 0, armed_v = 0;
+            uint32_t par_q = 0, par_k = 0, par_v = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
                 const UnitCoord c = decode_unit(p, u);
@@ -301,7 +379,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     const uint32_t sk = kt % KSTAGES, pk = (kt / KSTAGES) & 1;
                     if (!(ok = waiter.wait(bar(B_K_EMPTY + sk), pk ^ 1, ROLE_TMA))) break;
                     mbar_arrive_expect_tx(bar(B_K_FULL + sk), TILE_BYTES);
-                    armed_k[sk] = 1; par_k[sk] = pk;
+                    armed_k |= 1u << sk;
+                    par_k = (par_k & ~(1u << sk)) | (pk << sk);
                     for (int bx = 0; bx < 2; ++bx)
                         tma_load_4d(sK + sk * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + sk), bx * 64, c.h,
                                     j * BN, c.b);
@@ -309,7 +388,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     const uint32_t sv = vt % VSTAGES, pv = (vt / VSTAGES) & 1;
                     if (!(ok = waiter.wait(bar(B_V_EMPTY + sv), pv ^ 1, ROLE_TMA))) break;
                     mbar_arrive_expect_tx(bar(B_V_FULL + sv), TILE_BYTES);
-                    armed_v[sv] = 1; par_v[sv] = pv;
+                    armed_v |= 1u << sv;
+                    par_v = (par_v & ~(1u << sv)) | (pv << sv);
                     for (int bx = 0; bx < 2; ++bx)
                         tma_load_4d(sV + sv * TILE_BYTES + bx * BOX_BYTES, &p.tm_v, bar(B_V_FULL + sv), bx * 64, c.h,
                                     j * BN, c.b);
@@ -323,12 +403,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 Waiter tail{&never, 20000000ull};
                 if (armed_q) tail.wait(bar(B_Q_FULL), par_q, ROLE_TMA);
                 for (int s = 0; s < KSTAGES; ++s)
-                    if (armed_k[s]) tail.wait(bar(B_K_FULL + s), par_k[s], ROLE_TMA);
+                    if ((armed_k >> s) & 1u) tail.wait(bar(B_K_FULL + s), (par_k >> s) & 1u, ROLE_TMA);
                 for (int s = 0; s < VSTAGES; ++s)
-                    if (armed_v[s]) tail.wait(bar(B_V_FULL + s), par_v[s], ROLE_TMA);
+                    if ((armed_v >> s) & 1u) tail.wait(bar(B_V_FULL + s), (par_v >> s) & 1u, ROLE_TMA);
             }
         }
-    } else if (warp == WARP_MMA) {
+      } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
             uint32_t kt = 0, vt = 0, lu = 0;
@@ -390,29 +470,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 tail.wait(bar(B_DRAIN), 0, ROLE_MMA);
             }
         }
+      }
     } else if (warp >= WARP_ROPE) {
+        regs_decrease<REGS_ROPE>();
         // ------------------------------------------------------------ RoPE
         const int rt = threadIdx.x - WARP_ROPE * 32;
-        const RopeLane L = make_rope_lane(rt, p.theta_log2);
+        const RopeLane L = make_rope_lane(rt, p);
         uint32_t kt = 0, lu = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
             const UnitCoord c = decode_unit(p, u);
             if (!waiter.wait(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
             for (int qi = 0; qi < QTILES; ++qi)
-                rope_tile(sQ + qi * TILE_BYTES, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
+                rope_tile(sQ + qi * TILE_BYTES, sTable, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
             fence_proxy_async_smem();
             mbar_arrive(bar(B_Q_READY));
             bool ok = true;
             for (int j = 0; j < c.nt; ++j, ++kt) {
                 const uint32_t sk = kt % KSTAGES;
                 if (!(ok = waiter.wait(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
-                if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, j * BN, rt, L, p);
+                if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_K_READY + sk));
             }
             if (!ok) break;
         }
     } else {
+        regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
         const int qi = warp >> 2;                       // Q tile of this warpgroup
         const int row = ((warp & 3) << 5) + lane;       // = TMEM lane
@@ -429,51 +512,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             for (int j = 0; j < c.nt; ++j, ++sp) {
                 if (!(ok = waiter.wait_warp(bar(B_S_FULL + qi), sp & 1, ROLE_SOFTMAX))) break;
                 tc_fence_after();
-                const int lim = (j == c.nt - 1) ? c.last_lim : BN;
-                uint32_t r[32];
-                float mx = -INFINITY;
+                uint32_t sr[BN];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    tmem_ld32(tS + 32 * ch, r);
-                    tmem_wait_ld();
+                for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + 32 * ch, sr + 32 * ch);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float s = (32 * ch + e < lim) ? __uint_as_float(r[e]) : -INFINITY;
-                        mx = fmaxf(mx, s);
-                    }
+                for (int ch = 0; ch < BN / 32; ++ch) reg_fence32(sr + 32 * ch);
+                if (j == c.nt - 1) {
+                    // key mask: columns at or past N + valid in the last tile
+#pragma unroll
+                    for (int e = 0; e < BN; ++e)
+                        if (e >= c.last_lim) sr[e] = __float_as_uint(-INFINITY);
                 }
-                const float mx_s = mx * sl2;
+                float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+                float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+                for (int e = 4; e < BN; e += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(sr[e]));
+                    mx1 = fmaxf(mx1, __uint_as_float(sr[e + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(sr[e + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(sr[e + 3]));
+                }
+                const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
                 float m_new = m, alpha = 1.f;
                 if (mx_s - m > RESCALE_THRESHOLD) {
                     m_new = mx_s;
                     alpha = ex2_approx(m - m_new);
                 }
-                float rs = 0.f;
+                const float nm = -m_new;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    tmem_ld32(tS + 32 * ch, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int col = 32 * ch + 2 * e;
-                        const float p0 = (col < lim) ? ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -m_new)) : 0.f;
-                        const float p1 =
-                            (col + 1 < lim) ? ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -m_new)) : 0.f;
-                        rs += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tS + 16 * ch, pk);
+                for (int e = 0; e < BN; e += 4) {
+                    float x0, x1, x2, x3;
+                    ffma2(x0, x1, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, sl2, nm, nm);
+                    ffma2(x2, x3, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]), sl2, sl2, nm, nm);
+                    x0 = ex2_approx(x0);
+                    x1 = ex2_approx(x1);
+                    x2 = ex2_approx(x2);
+                    x3 = ex2_approx(x3);
+                    fadd2(a0, a1, a0, a1, x0, x1);
+                    fadd2(a2, a3, a2, a3, x2, x3);
+                    sr[e / 2] = pack_bf16x2(x0, x1);
+                    sr[e / 2 + 1] = pack_bf16x2(x2, x3);
                 }
-                l = l * alpha + rs;
+                tmem_st32(tS, sr);
+                tmem_st32(tS + 32, sr + 32);
+                l = l * alpha + ((a0 + a1) + (a2 + a3));
                 m = m_new;
                 if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
 #pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
                         tmem_ld32(tO + 32 * ch, r);
                         tmem_wait_ld();
+                        reg_fence32(r);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        for (int e = 0; e < 32; e += 2) {
+                            float y0, y1;
+                            fmul2(y0, y1, __uint_as_float(r[e]), __uint_as_float(r[e + 1]), alpha, alpha);
+                            r[e] = __float_as_uint(y0);
+                            r[e + 1] = __float_as_uint(y1);
+                        }
                         tmem_st32(tO + 32 * ch, r);
                     }
                 }
@@ -495,6 +594,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 uint32_t r[32];
                 tmem_ld32(tO + 32 * ch, r);
                 tmem_wait_ld();
+                reg_fence32(r);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -508,7 +608,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             tc_fence_before();
         }
     }
-
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -584,6 +683,14 @@ static DeviceInfo& device_info(int dev) {
         if (di.ok &&
             cudaFuncSetAttribute(hv_attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
                 cudaSuccess)
+            di.ok = 0;
+        // The warpgroups' setmaxnreg split adds up to exactly 512 threads x 128
+        // registers; a kernel launched with fewer would wait forever on the
+        // increase, so refuse to launch one.
+        cudaFuncAttributes fa;
+        if (di.ok && (cudaFuncGetAttributes(&fa, hv_attn_fwd_kernel) != cudaSuccess ||
+                      fa.numRegs * NUM_THREADS < static_cast<int>(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE +
+                                                                  128 * REGS_CONTROL)))
             di.ok = 0;
     }
     return di;
@@ -662,8 +769,10 @@ int hv_attn_forward(const void* q, const void* k, const void* v, void* out, int 
     prm->H = heads;
     prm->S = S;
     prm->N = static_cast<int>(n_video);
+    prm->T = T;
     prm->Hp = Hp;
     prm->Wp = Wp;
+    prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
     prm->HpWp = Hp * Wp;
     prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
     prm->units = static_cast<int>(units);
