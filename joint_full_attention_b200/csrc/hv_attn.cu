@@ -70,8 +70,8 @@ static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL <= N
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + QTILES * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
-// cos/sin table of the rotation angles: float2 (cos, sin) per (axis, position,
-// pair) = 8*T + 28*(Hp + Wp) entries, built once per CTA.
+// cos/sin table of the rotation angles: a cos and a sin per (axis, position,
+// pair) = 8*T + 28*(Hp + Wp) entries of 8 bytes, built once per CTA.
 constexpr int OFF_TABLE = OFF_V + VSTAGES * TILE_BYTES;
 constexpr int TABLE_MAX_ENTRIES = 4096;
 constexpr int OFF_BAR = OFF_TABLE + TABLE_MAX_ENTRIES * 8;
@@ -141,10 +141,13 @@ struct Waiter {
             }
         }
     }
-    // Warp-uniform version for roles that continue with warp-collective ops.
+    // Warp-wide version: lane 0 waits, the result is broadcast and the
+    // warp synchronises, so the other lanes are ordered after the wait
+    // without each polling the barrier.
     __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, uint32_t role) const {
-        const bool ok = wait(bar, parity, role);
-        return __all_sync(0xffffffffu, ok);
+        int ok = 1;
+        if ((threadIdx.x & 31) == 0) ok = wait(bar, parity, role) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
     }
 };
 
@@ -173,7 +176,7 @@ struct RopeLane {
     int box, cin, axis;
     int i0;            // first pair index of the chunk inside its axis segment
     int half_dim;      // pairs in the axis segment (8 or 28)
-    int table_base;    // first table entry of the axis segment
+    int table_base;    // first table float of the axis segment
     float freq[4];
 };
 
@@ -196,9 +199,9 @@ __device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
     if (ch0 < 16) {
         L.axis = 0; L.i0 = ch0 / 2; dax = 16; L.table_base = 0;
     } else if (ch0 < 72) {
-        L.axis = 1; L.i0 = (ch0 - 16) / 2; dax = 56; L.table_base = 8 * p.T;
+        L.axis = 1; L.i0 = (ch0 - 16) / 2; dax = 56; L.table_base = 16 * p.T;
     } else {
-        L.axis = 2; L.i0 = (ch0 - 72) / 2; dax = 56; L.table_base = 8 * p.T + 28 * p.Hp;
+        L.axis = 2; L.i0 = (ch0 - 72) / 2; dax = 56; L.table_base = 16 * p.T + 56 * p.Hp;
     }
     L.half_dim = dax / 2;
 #pragma unroll
@@ -206,22 +209,26 @@ __device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
     return L;
 }
 
-// Fill the (cos, sin) table: entry e of axis a at position pos and pair i
-// holds the rotation by pos * theta^(-2i/d_a).
-__device__ __forceinline__ void build_rope_table(float2* table, const Params& p) {
-    const int n_t = 8 * p.T, n_h = 28 * p.Hp, n_w = 28 * p.Wp;
-    for (int e = threadIdx.x; e < n_t + n_h + n_w; e += blockDim.x) {
-        int pos, i, dax;
-        if (e < n_t) {
-            pos = e / 8; i = e % 8; dax = 16;
-        } else if (e < n_t + n_h) {
-            pos = (e - n_t) / 28; i = (e - n_t) % 28; dax = 56;
+// Fill the rotation table. Per axis segment (pairs P = 8, 28, 28) and per
+// position pos it holds P cosines then P sines: float f = base + pos*2P + k
+// is cos (k < P) or sin (k >= P) of pos * theta^(-2i/d_a), i = k mod P.
+// Cosines and sines in separate runs let a chunk's four of each be read
+// with one 16-byte load, and neighbouring chunks hit neighbouring banks.
+__device__ __forceinline__ void build_rope_table(float* table, const Params& p) {
+    const int n_t = 16 * p.T, n_h = 56 * p.Hp, n_w = 56 * p.Wp;
+    for (int f = threadIdx.x; f < n_t + n_h + n_w; f += blockDim.x) {
+        int pos, k, half, dax;
+        if (f < n_t) {
+            pos = f / 16; k = f % 16; half = 8; dax = 16;
+        } else if (f < n_t + n_h) {
+            pos = (f - n_t) / 56; k = (f - n_t) % 56; half = 28; dax = 56;
         } else {
-            pos = (e - n_t - n_h) / 28; i = (e - n_t - n_h) % 28; dax = 56;
+            pos = (f - n_t - n_h) / 56; k = (f - n_t - n_h) % 56; half = 28; dax = 56;
         }
+        const int i = k < half ? k : k - half;
         float sn, cs;
         sincospif(static_cast<float>(pos) * axis_freq(i, dax, p.theta_log2) * kInvPi, &sn, &cs);
-        table[e] = make_float2(cs, sn);
+        table[f] = k < half ? cs : sn;
     }
 }
 
@@ -231,31 +238,78 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) 
     return pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
 }
 
+__device__ __forceinline__ uint4 rotate_chunk(uint4 d, uint4 c, uint4 sn) {
+    d.x = rotate_pair(d.x, __uint_as_float(c.x), __uint_as_float(sn.x));
+    d.y = rotate_pair(d.y, __uint_as_float(c.y), __uint_as_float(sn.y));
+    d.z = rotate_pair(d.z, __uint_as_float(c.z), __uint_as_float(sn.z));
+    d.w = rotate_pair(d.w, __uint_as_float(c.w), __uint_as_float(sn.w));
+    return d;
+}
+
+struct GridPos {
+    int t, h, w;
+};
+
+// Move a token 8 positions further along the flattened (t, h, w) grid.
+__device__ __forceinline__ void advance8(GridPos& g, const Params& p) {
+    g.w += 8;
+    while (g.w >= p.Wp) {
+        g.w -= p.Wp;
+        if (++g.h == p.Hp) {
+            g.h = 0;
+            ++g.t;
+        }
+    }
+}
+
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int rt, const RopeLane& L,
                                           const Params& p) {
     const int rb = rt >> 4;
     int n = n0 + rb;
     if (n >= p.N) return;
-    // (t, h, w) of row rb, then stepped by 8 rows at a time
-    int w = n % p.Wp;
+    GridPos g;
+    g.w = n % p.Wp;
     const int th = n / p.Wp;
-    int h = th % p.Hp;
-    int t = th / p.Hp;
+    g.h = th % p.Hp;
+    g.t = th / p.Hp;
+    const uint32_t row_base = tile + L.box * BOX_BYTES + ((L.cin ^ rb) << 4);   // (r & 7) == rb for r = rb + 8k
+    const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
+    const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
+    const int stride = 2 * L.half_dim;
+    if (p.use_table) {
+        // two rows (r, r + 8) per iteration so that their loads overlap
 #pragma unroll 1
-    for (int k = 0; k < BM / 8; ++k) {
-        const int r = rb + 8 * k;
-        const int pos = L.axis == 0 ? t : (L.axis == 1 ? h : w);
-        const uint32_t addr = tile + L.box * BOX_BYTES + r * 128 + ((L.cin ^ (r & 7)) << 4);
-        uint4 d = lds128(addr);
-        if (p.use_table) {
-            const uint32_t ta = table + 8u * static_cast<uint32_t>(L.table_base + pos * L.half_dim + L.i0);
-            const uint4 c01 = lds128(ta);
-            const uint4 c23 = lds128(ta + 16);
-            d.x = rotate_pair(d.x, __uint_as_float(c01.x), __uint_as_float(c01.y));
-            d.y = rotate_pair(d.y, __uint_as_float(c01.z), __uint_as_float(c01.w));
-            d.z = rotate_pair(d.z, __uint_as_float(c23.x), __uint_as_float(c23.y));
-            d.w = rotate_pair(d.w, __uint_as_float(c23.z), __uint_as_float(c23.w));
-        } else {
+        for (int r = rb; r < BM; r += 16) {
+            const int pos0 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
+            const bool has1 = n + 8 < p.N;
+            advance8(g, p);
+            const int pos1 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
+            const uint32_t a0 = row_base + r * 128;
+            const uint32_t a1 = a0 + 8 * 128;
+            const uint32_t t0 = tab + 4u * static_cast<uint32_t>(pos0 * stride);
+            const uint32_t t1 = tab + 4u * static_cast<uint32_t>(pos1 * stride);
+            const uint4 d0 = lds128(a0);
+            const uint4 c0 = lds128(t0);
+            const uint4 s0 = lds128(t0 + sin_off);
+            uint4 d1 = d0, c1 = c0, s1 = s0;
+            if (has1) {
+                d1 = lds128(a1);
+                c1 = lds128(t1);
+                s1 = lds128(t1 + sin_off);
+            }
+            sts128(a0, rotate_chunk(d0, c0, s0));
+            if (!has1) break;
+            sts128(a1, rotate_chunk(d1, c1, s1));
+            n += 16;
+            if (n >= p.N) break;   // rows only grow: the rest are text or past the end
+            advance8(g, p);
+        }
+    } else {
+#pragma unroll 1
+        for (int r = rb; r < BM; r += 8) {
+            const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
+            const uint32_t a = row_base + r * 128;
+            uint4 d = lds128(a);
             uint32_t wv[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -263,18 +317,10 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
                 sincospif(static_cast<float>(pos) * L.freq[q] * kInvPi, &sn, &cs);
                 wv[q] = rotate_pair(wv[q], cs, sn);
             }
-            d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        }
-        sts128(addr, d);
-        n += 8;
-        if (n >= p.N) break;  // rows only grow: the rest are text or past the end
-        w += 8;
-        while (w >= p.Wp) {
-            w -= p.Wp;
-            if (++h == p.Hp) {
-                h = 0;
-                ++t;
-            }
+            sts128(a, make_uint4(wv[0], wv[1], wv[2], wv[3]));
+            n += 8;
+            if (n >= p.N) break;
+            advance8(g, p);
         }
     }
 }
@@ -317,11 +363,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q_FULL), 1);
-        mbar_init(bar(B_Q_READY), ROPE_THREADS);
+        mbar_init(bar(B_Q_READY), ROPE_THREADS / 32);
         mbar_init(bar(B_Q_EMPTY), 1);
         for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(bar(B_K_FULL + s), 1);
-            mbar_init(bar(B_K_READY + s), ROPE_THREADS);
+            mbar_init(bar(B_K_READY + s), ROPE_THREADS / 32);
             mbar_init(bar(B_K_EMPTY + s), 1);
         }
         for (int s = 0; s < VSTAGES; ++s) {
@@ -330,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
         for (int i = 0; i < QTILES; ++i) {
             mbar_init(bar(B_S_FULL + i), 1);
-            mbar_init(bar(B_P_READY + i), 128);
+            mbar_init(bar(B_P_READY + i), 4);
             mbar_init(bar(B_O_DONE + i), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
@@ -341,7 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
-    if (p.use_table) build_rope_table(reinterpret_cast<float2*>(base_ptr + OFF_TABLE), p);
+    if (p.use_table) build_rope_table(reinterpret_cast<float*>(base_ptr + OFF_TABLE), p);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -479,18 +525,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         uint32_t kt = 0, lu = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
             const UnitCoord c = decode_unit(p, u);
-            if (!waiter.wait(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
+            if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
             for (int qi = 0; qi < QTILES; ++qi)
                 rope_tile(sQ + qi * TILE_BYTES, sTable, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
             fence_proxy_async_smem();
-            mbar_arrive(bar(B_Q_READY));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_Q_READY));
             bool ok = true;
             for (int j = 0; j < c.nt; ++j, ++kt) {
                 const uint32_t sk = kt % KSTAGES;
-                if (!(ok = waiter.wait(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
+                if (!(ok = waiter.wait_warp(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
                 if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
                 fence_proxy_async_smem();
-                mbar_arrive(bar(B_K_READY + sk));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_K_READY + sk));
             }
             if (!ok) break;
         }
@@ -578,7 +626,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar(B_P_READY + qi));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_P_READY + qi));
             }
             if (!ok) break;
             // epilogue: out = O / l as bf16, one 256-byte row per thread
