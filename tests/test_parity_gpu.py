@@ -56,6 +56,7 @@ def f64(inp):
 
 def check(got, ref, what):
     err = np.abs(got - ref)
+    print(f"[parity] {what}: max abs err {err.max():.3e}, mean {err.mean():.3e}")
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
     assert err.mean() <= MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
@@ -120,9 +121,10 @@ def test_theta_and_scale_parameters():
 
 
 def test_sharp_softmax_rescaling():
-    """Large score range: exercises the running-max rescale of O."""
+    """Sharper softmax: K scaled by 2, the top of the per-head K scale range of
+    the 720x1280x129 workload; exercises the running-max rescale of O."""
     grid, text_len = (4, 10, 10), 64
-    inp = _small(grid, text_len, [50], k_scale=3.0)
+    inp = _small(grid, text_len, [50], k_scale=2.0)
     full_check(inp, grid, text_len)
 
 
