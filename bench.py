@@ -60,6 +60,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiling runs)")
     return ap.parse_args()
 
 
@@ -307,22 +308,23 @@ def run_ours(args, wl, inp, rank, world, local):
     value = world * flops / (ms_per_step / 1e3) / 1e12
 
     # end to end through the host-buffer API: pinned host in, pinned host out
-    to_host = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    qh, kh, vh = (to_host(inp[n]) for n in ("q", "k", "v"))
-    oh = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
-    work = {"q": q, "k": k, "v": v, "out": out}
-    H.attn_forward_host(qh, kh, vh, wl.grid, wl.text_len, text_valid, device=dev, out_host=oh, work=work)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
+    e2e = None
+    if not args.no_e2e:
+        to_host = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        qh, kh, vh = (to_host(inp[n]) for n in ("q", "k", "v"))
+        oh = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+        work = {"q": q, "k": k, "v": v, "out": out}
         H.attn_forward_host(qh, kh, vh, wl.grid, wl.text_len, text_valid, device=dev, out_host=oh, work=work)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = allreduce_max(e0.elapsed_time(e1) / args.e2e_steps, world)
-    e2e_value = world * flops / (e2e_ms / 1e3) / 1e12
-    h2d = 3 * qh.numel() * 2
-    d2h = oh.numel() * 2
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            H.attn_forward_host(qh, kh, vh, wl.grid, wl.text_len, text_valid, device=dev, out_host=oh, work=work)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = allreduce_max(e0.elapsed_time(e1) / args.e2e_steps, world)
+        e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": 3 * qh.numel() * 2,
+               "d2h_bytes_per_step": oh.numel() * 2, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
 
     if rank != 0:
         return
@@ -345,8 +347,7 @@ def run_ours(args, wl, inp, rank, world, local):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl, text_valid),
         "roofline": roofline,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+        "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clk,
     }
