@@ -61,6 +61,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiling runs)")
+    ap.add_argument("--no-ws", action="store_true", help="skip timing the workspace (pre-rotated K) path")
     return ap.parse_args()
 
 
@@ -307,6 +308,30 @@ def run_ours(args, wl, inp, rank, world, local):
     ms_per_step = allreduce_max(total_ms / args.steps, world)
     value = world * flops / (ms_per_step / 1e3) / 1e12
 
+    # the workspace path: K rotated once by a memory-bound kernel, then attention
+    ws_line = None
+    if not args.no_ws:
+        ws = torch.empty(H.workspace_bytes(wl.batch, wl.heads, wl.grid, wl.text_len) // 2, dtype=torch.bfloat16,
+                         device=dev)
+        for _ in range(max(1, args.warmup)):
+            H.attn_forward_ws(q, k, v, wl.grid, wl.text_len, text_valid, out=out, workspace=ws, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record(stream)
+        for _ in range(args.steps):
+            H.attn_forward_ws(q, k, v, wl.grid, wl.text_len, text_valid, out=out, workspace=ws, stream=stream)
+        w1.record(stream)
+        torch.cuda.synchronize(dev)
+        if H.last_device_error() != 0:
+            raise RuntimeError("device error in the workspace path")
+        ws_ms = allreduce_max(w0.elapsed_time(w1) / args.steps, world)
+        ws_line = {"value": world * flops / (ws_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ws_ms,
+                   "gpu_launches_per_step": 2, "workspace_bytes": ws.numel() * 2,
+                   "what": "hv_attn_forward_ws: keys rotated once into a caller workspace by a memory-bound "
+                           "kernel, then the attention kernel rotating Q on load; output bit-identical"}
+        del ws
+
     # end to end through the host-buffer API: pinned host in, pinned host out
     e2e = None
     if not args.no_e2e:
@@ -350,6 +375,7 @@ def run_ours(args, wl, inp, rank, world, local):
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clk,
+        "workspace_path": ws_line,
     }
     if world == 1 and not args.no_cpu_baseline:
         cpu_value, info = oracle_sample(wl, inp, args.cpu_seconds)

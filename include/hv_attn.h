@@ -27,6 +27,8 @@
 #ifndef HV_ATTN_H
 #define HV_ATTN_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -42,7 +44,8 @@ enum hv_status {
     HV_ERR_BAD_SCALAR = 7,     /* rope_theta <= 0 or not finite, scale not finite    */
     HV_ERR_NO_DEVICE = 8,      /* current CUDA device is not an sm_100 (B200) part   */
     HV_ERR_LAUNCH = 9,         /* a CUDA runtime/driver call failed                  */
-    HV_ERR_DEVICE_TIMEOUT = 10 /* a kernel-side wait ran out (see hv_attn_last_device_error) */
+    HV_ERR_DEVICE_TIMEOUT = 10,/* a kernel-side wait ran out (see hv_attn_last_device_error) */
+    HV_ERR_WORKSPACE = 11      /* workspace NULL, not 16-byte aligned, too small or overlapping */
 };
 
 #define HV_HEAD_DIM 128
@@ -83,6 +86,35 @@ int hv_attn_forward(const void* q, const void* k, const void* v, void* out,
                     int B, int heads, int T, int Hp, int Wp,
                     int text_len, const int* text_valid,
                     float rope_theta, float scale, void* cuda_stream);
+
+/*
+ * hv_attn_forward_ws - the same result as hv_attn_forward, in two stages:
+ * a memory-bound kernel first writes the rotated keys R(K) (video rows
+ * rotated exactly as hv_attn_forward rotates them, text rows copied) into
+ * `workspace`, then the attention kernel reads them and rotates only Q as it
+ * loads it. The output is bit-identical to hv_attn_forward's. This trades
+ * workspace_bytes >= hv_attn_workspace_bytes(...) of device memory and one
+ * extra read and write of K (HBM traffic of 2 * B*S*heads*256 bytes) for
+ * taking the per-tile key rotation out of the attention loop (§5.5 "3D
+ * RoPE" applies R to K once; it does not say where).
+ *
+ * workspace: device pointer owned by the caller, 16-byte aligned, not
+ *            overlapping q, k, v or out; its contents on return are R(K).
+ * Other arguments, ownership, asynchrony and errors as hv_attn_forward;
+ * HV_ERR_WORKSPACE for a bad workspace. Two kernels are enqueued on the
+ * stream, in order.
+ */
+int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out,
+                       int B, int heads, int T, int Hp, int Wp,
+                       int text_len, const int* text_valid,
+                       float rope_theta, float scale,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * hv_attn_workspace_bytes - workspace hv_attn_forward_ws needs:
+ * B * (T*Hp*Wp + text_len) * heads * 128 * 2 bytes; -1 for a bad shape.
+ */
+long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len);
 
 /*
  * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)

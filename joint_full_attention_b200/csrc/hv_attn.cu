@@ -57,7 +57,11 @@ constexpr int NUM_THREADS = NUM_WARPS * 32;
 constexpr int WARP_ROPE = 8;
 constexpr int WARP_TMA = 12;
 constexpr int WARP_MMA = 13;
-constexpr int ROPE_THREADS = 128;
+// RoPE runs on warpgroup 2 (warps 8-11) and on the two control-warpgroup
+// warps that neither load nor issue MMAs (warps 14-15).
+constexpr int ROPE_THREADS = 192;
+constexpr int ROPE_WARPS = ROPE_THREADS / 32;
+constexpr int ROPE_GROUPS = ROPE_THREADS / 16;   // rows rb, rb + 12, rb + 24, ... per thread
 // per-thread registers after setmaxnreg: 2 x 128 x 176 + 128 x 64 + 128 x 96
 // = 65536 = 512 threads x 128 registers at launch
 constexpr uint32_t REGS_SOFTMAX = 176;
@@ -110,7 +114,8 @@ struct __align__(64) Params {
     CUtensorMap tm_v;
     __nv_bfloat16* out;
     int B, H, S, N, T, Hp, Wp, HpWp;
-    int use_table;      // 1: cos/sin from the shared-memory table, 0: sincosf per pair
+    int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
+    int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
     int n_qunits;       // ceil(S / 256)
     int units;          // B * H * n_qunits
     float theta_log2;   // log2(rope_theta)
@@ -177,7 +182,6 @@ struct RopeLane {
     int i0;            // first pair index of the chunk inside its axis segment
     int half_dim;      // pairs in the axis segment (8 or 28)
     int table_base;    // first table float of the axis segment
-    float freq[4];
 };
 
 // Angles are passed to sincospif in units of pi: sin(pi*x) needs no
@@ -186,7 +190,12 @@ constexpr float kInvPi = 0.318309886183790672f;
 
 __device__ __forceinline__ float axis_freq(int i, int dax, float theta_log2) {
     // theta^(-2i/d) = 2^(-(2i/d) * log2(theta))
-    return exp2f(-static_cast<float>(2 * i) * theta_log2 / static_cast<float>(dax));
+    return exp2f(__fdiv_rn(__fmul_rn(-static_cast<float>(2 * i), theta_log2), static_cast<float>(dax)));
+}
+
+// The angle pos * theta^(-2i/d) in units of pi, for sincospif.
+__device__ __forceinline__ float angle_over_pi(int pos, int i, int dax, float theta_log2) {
+    return __fmul_rn(__fmul_rn(static_cast<float>(pos), axis_freq(i, dax, theta_log2)), kInvPi);
 }
 
 __device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
@@ -204,8 +213,6 @@ __device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
         L.axis = 2; L.i0 = (ch0 - 72) / 2; dax = 56; L.table_base = 16 * p.T + 56 * p.Hp;
     }
     L.half_dim = dax / 2;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) L.freq[q] = axis_freq(L.i0 + q, dax, p.theta_log2);
     return L;
 }
 
@@ -227,16 +234,21 @@ __device__ __forceinline__ void build_rope_table(float* table, const Params& p) 
         }
         const int i = k < half ? k : k - half;
         float sn, cs;
-        sincospif(static_cast<float>(pos) * axis_freq(i, dax, p.theta_log2) * kInvPi, &sn, &cs);
+        sincospif(angle_over_pi(pos, i, dax, p.theta_log2), &sn, &cs);
         table[f] = k < half ? cs : sn;
     }
 }
 
+// Explicitly rounded operations (no contraction choices left to the
+// compiler), so that every kernel rotating a pair gets the same bits.
 __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
     const float x0 = __uint_as_float(w << 16);          // channel 2i   (low half)
     const float x1 = __uint_as_float(w & 0xFFFF0000u);  // channel 2i+1 (high half)
-    return pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+    const float y0 = __fmaf_rn(x0, cs, -__fmul_rn(x1, sn));
+    const float y1 = __fmaf_rn(x0, sn, __fmul_rn(x1, cs));
+    return pack_bf16x2(y0, y1);
 }
+
 
 __device__ __forceinline__ uint4 rotate_chunk(uint4 d, uint4 c, uint4 sn) {
     d.x = rotate_pair(d.x, __uint_as_float(c.x), __uint_as_float(sn.x));
@@ -250,9 +262,9 @@ struct GridPos {
     int t, h, w;
 };
 
-// Move a token 8 positions further along the flattened (t, h, w) grid.
+// Move a token ROPE_GROUPS positions further along the flattened (t, h, w) grid.
 __device__ __forceinline__ void advance8(GridPos& g, const Params& p) {
-    g.w += 8;
+    g.w += ROPE_GROUPS;
     while (g.w >= p.Wp) {
         g.w -= p.Wp;
         if (++g.h == p.Hp) {
@@ -272,20 +284,21 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
     const int th = n / p.Wp;
     g.h = th % p.Hp;
     g.t = th / p.Hp;
-    const uint32_t row_base = tile + L.box * BOX_BYTES + ((L.cin ^ rb) << 4);   // (r & 7) == rb for r = rb + 8k
+    const uint32_t box_base = tile + L.box * BOX_BYTES;
+    auto row_addr = [&](int r) { return box_base + r * 128 + ((L.cin ^ (r & 7)) << 4); };
     const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
     const int stride = 2 * L.half_dim;
     if (p.use_table) {
-        // two rows (r, r + 8) per iteration so that their loads overlap
+        // two rows (r, r + ROPE_GROUPS) per iteration so that their loads overlap
 #pragma unroll 1
-        for (int r = rb; r < BM; r += 16) {
+        for (int r = rb; r < BM; r += 2 * ROPE_GROUPS) {
             const int pos0 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
-            const bool has1 = n + 8 < p.N;
+            const bool has1 = n + ROPE_GROUPS < p.N && r + ROPE_GROUPS < BM;
             advance8(g, p);
             const int pos1 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
-            const uint32_t a0 = row_base + r * 128;
-            const uint32_t a1 = a0 + 8 * 128;
+            const uint32_t a0 = row_addr(r);
+            const uint32_t a1 = row_addr(r + ROPE_GROUPS);
             const uint32_t t0 = tab + 4u * static_cast<uint32_t>(pos0 * stride);
             const uint32_t t1 = tab + 4u * static_cast<uint32_t>(pos1 * stride);
             const uint4 d0 = lds128(a0);
@@ -300,28 +313,56 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
             sts128(a0, rotate_chunk(d0, c0, s0));
             if (!has1) break;
             sts128(a1, rotate_chunk(d1, c1, s1));
-            n += 16;
+            n += 2 * ROPE_GROUPS;
             if (n >= p.N) break;   // rows only grow: the rest are text or past the end
             advance8(g, p);
         }
     } else {
 #pragma unroll 1
-        for (int r = rb; r < BM; r += 8) {
+        for (int r = rb; r < BM; r += ROPE_GROUPS) {
             const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
-            const uint32_t a = row_base + r * 128;
+            const uint32_t a = row_addr(r);
             uint4 d = lds128(a);
             uint32_t wv[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float sn, cs;
-                sincospif(static_cast<float>(pos) * L.freq[q] * kInvPi, &sn, &cs);
+                sincospif(angle_over_pi(pos, L.i0 + q, 2 * L.half_dim, p.theta_log2), &sn, &cs);
                 wv[q] = rotate_pair(wv[q], cs, sn);
             }
             sts128(a, make_uint4(wv[0], wv[1], wv[2], wv[3]));
-            n += 8;
+            n += ROPE_GROUPS;
             if (n >= p.N) break;
             advance8(g, p);
         }
+    }
+}
+
+// The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
+// each to the MMA warp.
+__device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
+                                          uint32_t sK, uint32_t sTable) {
+    const RopeLane L = make_rope_lane(rt, p);
+    const int lane = threadIdx.x & 31;
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t kt = 0, lu = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
+        const UnitCoord c = decode_unit(p, u);
+        if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
+        for (int qi = 0; qi < QTILES; ++qi) rope_tile(sQ + qi * TILE_BYTES, sTable, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_Q_READY));
+        bool ok = true;
+        for (int j = 0; j < c.nt; ++j, ++kt) {
+            const uint32_t sk = kt % KSTAGES;
+            if (!(ok = waiter.wait_warp(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
+            if (!p.k_rotated && j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_K_READY + sk));
+        }
+        if (!ok) break;
     }
 }
 
@@ -363,11 +404,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q_FULL), 1);
-        mbar_init(bar(B_Q_READY), ROPE_THREADS / 32);
+        mbar_init(bar(B_Q_READY), ROPE_WARPS);
         mbar_init(bar(B_Q_EMPTY), 1);
         for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(bar(B_K_FULL + s), 1);
-            mbar_init(bar(B_K_READY + s), ROPE_THREADS / 32);
+            mbar_init(bar(B_K_READY + s), ROPE_WARPS);
             mbar_init(bar(B_K_EMPTY + s), 1);
         }
         for (int s = 0; s < VSTAGES; ++s) {
@@ -454,6 +495,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     if ((armed_v >> s) & 1u) tail.wait(bar(B_V_FULL + s), (par_v >> s) & 1u, ROLE_TMA);
             }
         }
+      } else if (warp > WARP_MMA) {
+        // RoPE helpers: threads 128..191 of the RoPE role
+        rope_role(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
@@ -520,28 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     } else if (warp >= WARP_ROPE) {
         regs_decrease<REGS_ROPE>();
         // ------------------------------------------------------------ RoPE
-        const int rt = threadIdx.x - WARP_ROPE * 32;
-        const RopeLane L = make_rope_lane(rt, p);
-        uint32_t kt = 0, lu = 0;
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
-            const UnitCoord c = decode_unit(p, u);
-            if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
-            for (int qi = 0; qi < QTILES; ++qi)
-                rope_tile(sQ + qi * TILE_BYTES, sTable, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_Q_READY));
-            bool ok = true;
-            for (int j = 0; j < c.nt; ++j, ++kt) {
-                const uint32_t sk = kt % KSTAGES;
-                if (!(ok = waiter.wait_warp(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
-                if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_K_READY + sk));
-            }
-            if (!ok) break;
-        }
+        rope_role(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -663,6 +686,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     if (warp == WARP_MMA) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// Workspace path, first stage: K' = R(K) for every video row, other rows
+// copied, [B, S, heads, 128] bf16 in and out. One thread per 16-byte chunk
+// (four adjacent channel pairs of one axis segment); the same fp32 rotation
+// and bf16 rounding as the attention kernel's in-shared-memory path, with
+// (cos, sin) from sincospif of the same angles, so both paths agree bit for
+// bit. Memory-bound: reads and writes B*S*heads*256 bytes once.
+__global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict__ kin, uint4* __restrict__ kout,
+                                                        long long n_chunks, int H, int S, int N, int Hp, int Wp,
+                                                        float theta_log2) {
+    const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_chunks; e += step) {
+        uint4 d = __ldg(kin + e);
+        const int cc = static_cast<int>(e & 15);
+        const long long row = e >> 4;               // (b * S + s) * H + h
+        const int s_idx = static_cast<int>((row / H) % S);
+        if (s_idx < N) {
+            const int ch0 = cc * 8;
+            int i0, dax, pos;
+            if (ch0 < 16) {
+                i0 = ch0 / 2; dax = 16; pos = s_idx / (Hp * Wp);
+            } else if (ch0 < 72) {
+                i0 = (ch0 - 16) / 2; dax = 56; pos = (s_idx / Wp) % Hp;
+            } else {
+                i0 = (ch0 - 72) / 2; dax = 56; pos = s_idx % Wp;
+            }
+            uint32_t wv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float sn, cs;
+                sincospif(angle_over_pi(pos, i0 + q, dax, theta_log2), &sn, &cs);
+                wv[q] = rotate_pair(wv[q], cs, sn);
+            }
+            d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        kout[e] = d;
+    }
+}
+
 // One warp waits on an mbarrier that nothing completes; the bounded wait must
 // run out, record ROLE_SELFTEST and return.
 __global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns) {
@@ -752,6 +813,78 @@ static bool overlaps(const void* a, const void* b, size_t bytes) {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 
+struct Call {
+    int S = 0, N = 0, sms = 0;
+    long long units = 0;
+    size_t bytes = 0;   // bytes of one [B, S, heads, 128] bf16 tensor
+};
+
+static int validate(const void* q, const void* k, const void* v, const void* out, int B, int heads, int T, int Hp,
+                    int Wp, int text_len, const int* text_valid, float rope_theta, float scale, Call& call) {
+    if (!q || !k || !v || !out || !text_valid) return HV_ERR_NULL_POINTER;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+    if (mis & 15u) return HV_ERR_MISALIGNED;
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH) return HV_ERR_BAD_SHAPE;
+    if (text_len < 0 || text_len > HV_MAX_TEXT_LEN) return HV_ERR_BAD_TEXT;
+    for (int b = 0; b < B; ++b)
+        if (text_valid[b] < 0 || text_valid[b] > text_len) return HV_ERR_BAD_TEXT;
+    if (!std::isfinite(rope_theta) || !(rope_theta > 0.f) || !std::isfinite(scale)) return HV_ERR_BAD_SCALAR;
+    const long long n_video = static_cast<long long>(T) * Hp * Wp;
+    const long long s_len = n_video + text_len;
+    const long long units = static_cast<long long>(B) * heads * ((s_len + UNIT_ROWS - 1) / UNIT_ROWS);
+    if (s_len + UNIT_ROWS >= (1ll << 31) || s_len * heads * D >= (1ll << 31) || units >= (1ll << 31))
+        return HV_ERR_TOO_LARGE;
+    const size_t bytes = static_cast<size_t>(B) * s_len * heads * D * 2;
+    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return HV_ERR_ALIAS;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    DeviceInfo& di = device_info(dev);
+    if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    call.S = static_cast<int>(s_len);
+    call.N = static_cast<int>(n_video);
+    call.sms = di.sms;
+    call.units = units;
+    call.bytes = bytes;
+    return HV_OK;
+}
+
+static int launch_attention(const Call& call, const void* q, const void* k, const void* v, void* out, int B,
+                            int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
+                            float scale, bool k_rotated, cudaStream_t stream) {
+    (void)text_len;
+    Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
+    std::memset(prm, 0, sizeof(Params));
+    const int S = call.S;
+    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, S, heads) ||
+        !make_qkv_map(&prm->tm_v, v, B, S, heads)) {
+        delete prm;
+        return HV_ERR_LAUNCH;
+    }
+    prm->out = static_cast<__nv_bfloat16*>(out);
+    prm->B = B;
+    prm->H = heads;
+    prm->S = S;
+    prm->N = call.N;
+    prm->T = T;
+    prm->Hp = Hp;
+    prm->Wp = Wp;
+    prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
+    prm->k_rotated = k_rotated ? 1 : 0;
+    prm->HpWp = Hp * Wp;
+    prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
+    prm->units = static_cast<int>(call.units);
+    prm->theta_log2 = static_cast<float>(std::log2(static_cast<double>(rope_theta)));
+    prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    prm->timeout_ns = kWaitTimeoutNs;
+    for (int b = 0; b < B; ++b) prm->text_valid[b] = text_valid[b];
+    const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
+    hv_attn_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    delete prm;
+    const cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
+}
+
 }  // namespace hv
 
 extern "C" {
@@ -769,6 +902,7 @@ const char* hv_attn_status_string(int status) {
         case HV_ERR_NO_DEVICE: return "current CUDA device is not sm_100";
         case HV_ERR_LAUNCH: return "CUDA launch or driver call failed";
         case HV_ERR_DEVICE_TIMEOUT: return "a kernel-side wait timed out";
+        case HV_ERR_WORKSPACE: return "workspace missing, misaligned, too small or overlapping an operand";
         default: return "unknown status";
     }
 }
@@ -783,58 +917,39 @@ long long hv_video_tokens(int frames, int height, int width) {
 int hv_attn_forward(const void* q, const void* k, const void* v, void* out, int B, int heads, int T, int Hp, int Wp,
                     int text_len, const int* text_valid, float rope_theta, float scale, void* cuda_stream) {
     using namespace hv;
-    if (!q || !k || !v || !out || !text_valid) return HV_ERR_NULL_POINTER;
-    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
-    if (mis & 15u) return HV_ERR_MISALIGNED;
-    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH) return HV_ERR_BAD_SHAPE;
-    if (text_len < 0 || text_len > HV_MAX_TEXT_LEN) return HV_ERR_BAD_TEXT;
-    for (int b = 0; b < B; ++b)
-        if (text_valid[b] < 0 || text_valid[b] > text_len) return HV_ERR_BAD_TEXT;
-    if (!std::isfinite(rope_theta) || !(rope_theta > 0.f) || !std::isfinite(scale)) return HV_ERR_BAD_SCALAR;
-    const long long n_video = static_cast<long long>(T) * Hp * Wp;
-    const long long s_len = n_video + text_len;
-    const long long units = static_cast<long long>(B) * heads * ((s_len + UNIT_ROWS - 1) / UNIT_ROWS);
-    if (s_len + UNIT_ROWS >= (1ll << 31) || s_len * heads * D >= (1ll << 31) || units >= (1ll << 31))
-        return HV_ERR_TOO_LARGE;
-    const size_t bytes = static_cast<size_t>(B) * s_len * heads * D * 2;
-    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return HV_ERR_ALIAS;
+    Call call;
+    int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call);
+    if (st != HV_OK) return st;
+    return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false,
+                            static_cast<cudaStream_t>(cuda_stream));
+}
 
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
-    DeviceInfo& di = device_info(dev);
-    if (di.ok != 1) return HV_ERR_NO_DEVICE;
+long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len) {
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || text_len < 0 || text_len > HV_MAX_TEXT_LEN) return -1;
+    const long long s_len = static_cast<long long>(T) * Hp * Wp + text_len;
+    return static_cast<long long>(B) * s_len * heads * hv::D * 2;
+}
 
-    Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
-    std::memset(prm, 0, sizeof(Params));
-    const int S = static_cast<int>(s_len);
-    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, S, heads) ||
-        !make_qkv_map(&prm->tm_v, v, B, S, heads)) {
-        delete prm;
-        return HV_ERR_LAUNCH;
-    }
-    prm->out = static_cast<__nv_bfloat16*>(out);
-    prm->B = B;
-    prm->H = heads;
-    prm->S = S;
-    prm->N = static_cast<int>(n_video);
-    prm->T = T;
-    prm->Hp = Hp;
-    prm->Wp = Wp;
-    prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
-    prm->HpWp = Hp * Wp;
-    prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
-    prm->units = static_cast<int>(units);
-    prm->theta_log2 = static_cast<float>(std::log2(static_cast<double>(rope_theta)));
-    prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    prm->timeout_ns = kWaitTimeoutNs;
-    for (int b = 0; b < B; ++b) prm->text_valid[b] = text_valid[b];
-
-    const int grid = static_cast<int>(units < di.sms ? units : di.sms);
-    hv_attn_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, static_cast<cudaStream_t>(cuda_stream)>>>(*prm);
-    delete prm;
-    const cudaError_t err = cudaGetLastError();
-    return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
+int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out, int B, int heads, int T, int Hp,
+                       int Wp, int text_len, const int* text_valid, float rope_theta, float scale, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
+    using namespace hv;
+    Call call;
+    int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call);
+    if (st != HV_OK) return st;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) || workspace_bytes < call.bytes ||
+        overlaps(workspace, q, call.bytes) || overlaps(workspace, k, call.bytes) || overlaps(workspace, v, call.bytes) ||
+        overlaps(workspace, out, call.bytes))
+        return HV_ERR_WORKSPACE;
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const long long n_chunks = static_cast<long long>(call.bytes / 16);
+    const int grid = 8 * call.sms;
+    hv_rope_k_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<uint4*>(workspace), n_chunks,
+                                               heads, call.S, call.N, Hp, Wp,
+                                               static_cast<float>(std::log2(static_cast<double>(rope_theta))));
+    if (cudaGetLastError() != cudaSuccess) return HV_ERR_LAUNCH;
+    return launch_attention(call, q, workspace, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
+                            true, stream);
 }
 
 int hv_attn_last_device_error(void) {

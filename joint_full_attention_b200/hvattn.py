@@ -21,10 +21,10 @@ HV_OK = 0
 STATUS_NAMES = {
     0: "HV_OK", 1: "HV_ERR_NULL_POINTER", 2: "HV_ERR_MISALIGNED", 3: "HV_ERR_BAD_SHAPE",
     4: "HV_ERR_BAD_TEXT", 5: "HV_ERR_TOO_LARGE", 6: "HV_ERR_ALIAS", 7: "HV_ERR_BAD_SCALAR",
-    8: "HV_ERR_NO_DEVICE", 9: "HV_ERR_LAUNCH", 10: "HV_ERR_DEVICE_TIMEOUT",
+    8: "HV_ERR_NO_DEVICE", 9: "HV_ERR_LAUNCH", 10: "HV_ERR_DEVICE_TIMEOUT", 11: "HV_ERR_WORKSPACE",
 }
-EXPORTED = ("hv_attn_forward", "hv_video_tokens", "hv_attn_last_device_error",
-            "hv_attn_selftest_timeout", "hv_attn_status_string")
+EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_workspace_bytes", "hv_video_tokens",
+            "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
 
 
 class HVError(RuntimeError):
@@ -43,6 +43,12 @@ def lib() -> ctypes.CDLL:
         L.hv_attn_forward.restype = ctypes.c_int
         L.hv_attn_forward.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
             ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
+        L.hv_attn_forward_ws.restype = ctypes.c_int
+        L.hv_attn_forward_ws.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
+            ctypes.c_void_p]
+        L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
+        L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
         L.hv_video_tokens.argtypes = [ctypes.c_int] * 3
         L.hv_attn_last_device_error.restype = ctypes.c_int
@@ -111,6 +117,50 @@ def attn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_l
                                    ctypes.c_void_p(stream.cuda_stream))
     if st != HV_OK:
         raise HVError(st, "hv_attn_forward")
+    return out
+
+
+def workspace_bytes(batch: int, heads: int, grid, text_len: int) -> int:
+    """Device bytes ``attn_forward_ws`` needs for its rotated-key workspace."""
+    t_lat, hp, wp = (int(x) for x in grid)
+    return int(lib().hv_attn_workspace_bytes(int(batch), int(heads), t_lat, hp, wp, int(text_len)))
+
+
+def attn_forward_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, text_valid,
+                    rope_theta: float = 256.0, scale: float | None = None, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Same result as ``attn_forward``, keys pre-rotated once into ``workspace``.
+
+    ``workspace`` is any CUDA tensor of at least ``workspace_bytes(...)``
+    bytes (allocated here if None); on return it holds the rotated keys.
+    """
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    b_sz, _, heads, _ = q.shape
+    t_lat, hp, wp = (int(x) for x in grid)
+    if len(text_valid) != b_sz:
+        raise ValueError("text_valid needs one entry per batch sample")
+    need = workspace_bytes(b_sz, heads, grid, text_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 0) // 2, dtype=torch.bfloat16, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    valid = (ctypes.c_int * b_sz)(*[int(x) for x in text_valid])
+    if scale is None:
+        scale = 1.0 / math.sqrt(128)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = lib().hv_attn_forward_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b_sz, heads,
+                                      t_lat, hp, wp, int(text_len), valid, float(rope_theta), float(scale),
+                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                      ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_forward_ws")
     return out
 
 

@@ -89,6 +89,18 @@ def test_argument_validation_codes(lib):
     assert _call(lib, q=big, k=big * 2, v=big * 3, out=big + 4096) == 6
 
 
+def test_workspace_entry_points(lib):
+    assert lib.hv_attn_workspace_bytes(1, 24, 33, 45, 80, 256) == 119056 * 24 * 256
+    assert lib.hv_attn_workspace_bytes(2, 2, 2, 4, 4, 8) == 2 * 40 * 2 * 256
+    assert lib.hv_attn_workspace_bytes(0, 2, 2, 4, 4, 8) == -1
+    assert lib.hv_attn_workspace_bytes(1, 2, 2, 4, 4, 300) == -1
+    valid = (ctypes.c_int * 1)(5)
+    f = lib.hv_attn_forward_ws
+    # argument errors come first, before the workspace is looked at
+    assert f(None, 0x20000, 0x30000, 0x40000, 1, 2, 2, 4, 4, 8, valid, 256.0, 0.088, 0x90000, 1 << 20, None) == 1
+    assert f(0x10000, 0x20000, 0x30000, 0x40000, 0, 2, 2, 4, 4, 8, valid, 256.0, 0.088, 0x90000, 1 << 20, None) == 3
+
+
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     import torch
     if torch.cuda.is_available():

@@ -178,3 +178,61 @@ def test_bounded_wait_times_out_cleanly():
     # the context is still usable
     inp = _small((2, 4, 4), 8, [5])
     full_check(inp, (2, 4, 4), 8)
+
+
+# ------------------------------------------------ workspace (pre-rotated K) path
+
+def _run_both(inp, grid, text_len, theta=256.0):
+    q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
+    fused = H.attn_forward(q, k, v, grid, text_len, inp["text_valid"], theta)
+    ws = torch.empty(H.workspace_bytes(q.shape[0], q.shape[2], grid, text_len) // 2, dtype=torch.bfloat16,
+                     device="cuda")
+    two = H.attn_forward_ws(q, k, v, grid, text_len, inp["text_valid"], theta, workspace=ws)
+    torch.cuda.synchronize()
+    assert H.last_device_error() == 0
+    return fused, two, ws
+
+
+@pytest.mark.parametrize("name", ["tiny", "img256", "v544x960x17", "v720x1280x129"])
+def test_workspace_path_bit_identical(name):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, seed=4)
+    fused, two, _ = _run_both(inp, wl.grid, wl.text_len)
+    assert torch.equal(fused, two)
+
+
+@pytest.mark.parametrize("grid,text_len,valid", [((1, 1, 1), 0, [0]), ((5, 3, 11), 100, [1]),
+                                                 ((4, 8, 9), 19, [19, 3, 0])])
+def test_workspace_path_edge_shapes(grid, text_len, valid):
+    inp = _small(grid, text_len, valid, batch=len(valid))
+    fused, two, _ = _run_both(inp, grid, text_len, theta=1000.0)
+    assert torch.equal(fused, two)
+
+
+def test_workspace_holds_rotated_keys():
+    """The first stage writes R(K): video rows rotated (bf16 of the exact
+    rotation, within one bf16 step), text rows copied bit for bit."""
+    grid, text_len = (3, 5, 7), 24
+    inp = _small(grid, text_len, [9], heads=2)
+    _, _, ws = _run_both(inp, grid, text_len)
+    n = 105
+    got = ws.view(1, n + text_len, 2, 128).float().cpu().numpy().astype(np.float64)
+    k = W.bf16_bits_to_f64(inp["k"])
+    for h in range(2):
+        exact = O.rope3d_rotate(k[0, :n, h], O.token_positions(*grid))
+        # one bf16 step of the result, plus fp32 rounding of the rotation itself
+        step = np.abs(exact) * 2.0 ** -7 + 1e-5
+        assert np.all(np.abs(got[0, :n, h] - exact) <= step)
+        assert np.array_equal(got[0, n:, h], k[0, n:, h])
+
+
+def test_workspace_errors():
+    q = torch.zeros(1, 40, 2, 128, dtype=torch.bfloat16, device="cuda")
+    small = torch.empty(100, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward_ws(q, q, q, (2, 4, 4), 8, [5], workspace=small)
+    assert e.value.status == 11
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward_ws(q, q, q, (2, 4, 4), 8, [5], out=torch.empty_like(q), workspace=q.view(-1))
+    assert e.value.status == 11
+    assert H.last_device_error() == 0
