@@ -45,7 +45,8 @@ enum hv_status {
     HV_ERR_NO_DEVICE = 8,      /* current CUDA device is not an sm_100 (B200) part   */
     HV_ERR_LAUNCH = 9,         /* a CUDA runtime/driver call failed                  */
     HV_ERR_DEVICE_TIMEOUT = 10,/* a kernel-side wait ran out (see hv_attn_last_device_error) */
-    HV_ERR_WORKSPACE = 11      /* workspace NULL, not 16-byte aligned, too small or overlapping */
+    HV_ERR_WORKSPACE = 11,     /* workspace NULL, not 16-byte aligned, too small or overlapping */
+    HV_ERR_NOALLOC_LIMIT = 12  /* problem too large for hv_attn_forward_noalloc's built-in scratch */
 };
 
 #define HV_HEAD_DIM 128
@@ -115,6 +116,35 @@ int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out,
  * B * (T*Hp*Wp + text_len) * heads * 128 * 2 bytes; -1 for a bad shape.
  */
 long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len);
+
+/*
+ * hv_attn_forward_noalloc - hv_attn_forward_ws with no workspace argument and
+ * no allocation: the rotated keys go to a scratch array built into the
+ * library (HV_NOALLOC_MAX_BYTES = 64 MiB of device memory per device that
+ * loads the library, held until the process exits).
+ *
+ * No counterpart in the paper: this entry point exists for callers that
+ * cannot allocate device memory when they call attention - for example an
+ * application whose own allocator owns the device memory and forbids other
+ * allocations, or a tight loop that must not pay for cudaMalloc's implicit
+ * synchronisation - and that have no spare buffer to hand in as workspace.
+ *
+ * Arguments, result (bit-identical to hv_attn_forward) and errors as
+ * hv_attn_forward. Problems needing more than HV_NOALLOC_MAX_BYTES of
+ * rotated keys (B * S * heads * 256 bytes) are rejected with
+ * HV_ERR_NOALLOC_LIMIT before anything is launched. It calls no cudaMalloc,
+ * cudaFree or other allocating routine. The first call on a device looks up
+ * the scratch array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture. Every call on a
+ * device shares the one scratch array, which keeps the last call's contents:
+ * calls whose kernels overlap on the GPU (different streams, or different
+ * host threads) race on it and must be ordered by the caller.
+ */
+#define HV_NOALLOC_MAX_BYTES (64ull << 20)
+int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out,
+                            int B, int heads, int T, int Hp, int Wp,
+                            int text_len, const int* text_valid,
+                            float rope_theta, float scale, void* cuda_stream);
 
 /*
  * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)

@@ -849,6 +849,27 @@ static int validate(const void* q, const void* k, const void* v, const void* out
     return HV_OK;
 }
 
+// Built-in scratch for hv_attn_forward_noalloc: room for the rotated keys of
+// problems up to HV_NOALLOC_MAX_BYTES. It is part of the module, so every
+// device that loads this library holds it until the process exits; no
+// allocation call ever creates it. All calls share it.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HV_NOALLOC_MAX_BYTES];
+
+// Device address of g_noalloc_scratch on device `dev` (which must be the
+// current device), looked up once per device and then cached. In host code
+// the array's name is only a stand-in; the address must come from the runtime.
+static void* noalloc_scratch(int dev) {
+    static void* addr[64] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev & 63]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev & 63] = ptr;
+    }
+    return addr[dev & 63];
+}
+
 static int launch_attention(const Call& call, const void* q, const void* k, const void* v, void* out, int B,
                             int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
                             float scale, bool k_rotated, cudaStream_t stream) {
@@ -903,6 +924,8 @@ const char* hv_attn_status_string(int status) {
         case HV_ERR_LAUNCH: return "CUDA launch or driver call failed";
         case HV_ERR_DEVICE_TIMEOUT: return "a kernel-side wait timed out";
         case HV_ERR_WORKSPACE: return "workspace missing, misaligned, too small or overlapping an operand";
+        case HV_ERR_NOALLOC_LIMIT:
+            return "problem needs more scratch than hv_attn_forward_noalloc's built-in HV_NOALLOC_MAX_BYTES";
         default: return "unknown status";
     }
 }
@@ -949,6 +972,30 @@ int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out, i
                                                static_cast<float>(std::log2(static_cast<double>(rope_theta))));
     if (cudaGetLastError() != cudaSuccess) return HV_ERR_LAUNCH;
     return launch_attention(call, q, workspace, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
+                            true, stream);
+}
+
+int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int heads, int T,
+                            int Hp, int Wp, int text_len, const int* text_valid, float rope_theta, float scale,
+                            void* cuda_stream) {
+    using namespace hv;
+    Call call;
+    int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call);
+    if (st != HV_OK) return st;
+    if (call.bytes > HV_NOALLOC_MAX_BYTES) return HV_ERR_NOALLOC_LIMIT;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    void* scratch = noalloc_scratch(dev);
+    if (!scratch) return HV_ERR_LAUNCH;
+    // the first stage overwrites every byte of the scratch it uses, so
+    // nothing left there by an earlier call needs clearing
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const long long n_chunks = static_cast<long long>(call.bytes / 16);
+    hv_rope_k_kernel<<<8 * call.sms, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<uint4*>(scratch),
+                                                       n_chunks, heads, call.S, call.N, Hp, Wp,
+                                                       static_cast<float>(std::log2(static_cast<double>(rope_theta))));
+    if (cudaGetLastError() != cudaSuccess) return HV_ERR_LAUNCH;
+    return launch_attention(call, q, scratch, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
                             true, stream);
 }
 

@@ -22,8 +22,10 @@ STATUS_NAMES = {
     0: "HV_OK", 1: "HV_ERR_NULL_POINTER", 2: "HV_ERR_MISALIGNED", 3: "HV_ERR_BAD_SHAPE",
     4: "HV_ERR_BAD_TEXT", 5: "HV_ERR_TOO_LARGE", 6: "HV_ERR_ALIAS", 7: "HV_ERR_BAD_SCALAR",
     8: "HV_ERR_NO_DEVICE", 9: "HV_ERR_LAUNCH", 10: "HV_ERR_DEVICE_TIMEOUT", 11: "HV_ERR_WORKSPACE",
+    12: "HV_ERR_NOALLOC_LIMIT",
 }
-EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_workspace_bytes", "hv_video_tokens",
+EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", "hv_attn_workspace_bytes",
+            "hv_video_tokens",
             "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
 
 
@@ -47,6 +49,9 @@ def lib() -> ctypes.CDLL:
         L.hv_attn_forward_ws.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
             ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
             ctypes.c_void_p]
+        L.hv_attn_forward_noalloc.restype = ctypes.c_int
+        L.hv_attn_forward_noalloc.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
         L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
