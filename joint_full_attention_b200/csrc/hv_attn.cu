@@ -11,11 +11,11 @@
 // tile. Per CTA (one per SM, 512 threads = 4 warpgroups):
 //   warps 0-3   softmax for Q tile 0 (thread = TMEM lane = query row)
 //   warps 4-7   softmax for Q tile 1
-//   warps 8-11  RoPE: rotate the video rows of each Q/K tile in shared memory
-//               right after TMA lands it, then hand it to the tensor core
+//   warps 8-11, 14-15  RoPE: rotate the video rows of each Q/K tile in shared
+//               memory right after TMA lands it, then hand it to the tensor
+//               core (Q only when the keys arrive rotated)
 //   warp  12    TMA producer (Q once per unit, then K/V tiles into a ring)
 //   warp  13    TMEM owner and tcgen05.mma issuer
-//   warps 14-15 idle (complete the last warpgroup)
 // setmaxnreg moves registers to the softmax warpgroups, which hold a full
 // 128-column score row per thread.
 // Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the
@@ -354,10 +354,11 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_Q_READY));
         bool ok = true;
+        if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
         for (int j = 0; j < c.nt; ++j, ++kt) {
             const uint32_t sk = kt % KSTAGES;
             if (!(ok = waiter.wait_warp(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
-            if (!p.k_rotated && j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
+            if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_K_READY + sk));
@@ -501,6 +502,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
+            // K tiles are ready for the tensor core once the RoPE warps have
+            // rotated them, or, when they arrive rotated, once TMA lands them.
+            const int k_ready = p.k_rotated ? B_K_FULL : B_K_READY;
             uint32_t kt = 0, vt = 0, lu = 0;
             uint32_t pr[QTILES] = {0, 0};
             bool ok = true;
@@ -508,7 +512,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 const UnitCoord c = decode_unit(p, u);
                 if (!(ok = waiter.wait(bar(B_Q_READY), lu & 1, ROLE_MMA))) break;
                 uint32_t sk = kt % KSTAGES;
-                if (!(ok = waiter.wait(bar(B_K_READY + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                if (!(ok = waiter.wait(bar(k_ready + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
                 tc_fence_after();
                 issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
                 mma_commit(bar(B_S_FULL + 0));
@@ -530,7 +534,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     const bool more = j + 1 < c.nt;
                     sk = kt % KSTAGES;
                     if (more) {
-                        if (!(ok = waiter.wait(bar(B_K_READY + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                        if (!(ok = waiter.wait(bar(k_ready + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
                         tc_fence_after();
                         issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
                         mma_commit(bar(B_S_FULL + 0));

@@ -57,6 +57,14 @@ WORKLOADS: dict[str, Workload] = {
     "v544x960x129": Workload("v544x960x129", "544x960x129 video", 1, 24, (33, 34, 60), 256, full_check=False),
     "v720x1280x129": Workload("v720x1280x129", "720x1280x129 video", 1, 24, (33, 45, 80), 256,
                               k_head_scale=True, full_check=False),
+    # other supported sizes of the README's table (same ~118k-token scale, other aspect ratios)
+    "v960x960x129": Workload("v960x960x129", "960x960x129 video", 1, 24, (33, 60, 60), 256, full_check=False),
+    "v1104x832x129": Workload("v1104x832x129", "1104x832x129 video", 1, 24, (33, 69, 52), 256,
+                              full_check=False),
+    # two-branch classifier-free guidance: conditional and unconditional prompts
+    # batched together, each with its own valid text length
+    "cfg544x960x129": Workload("cfg544x960x129", "544x960x129 video, B=2 (CFG pair)", 2, 24, (33, 34, 60), 256,
+                               full_check=False),
 }
 
 BENCH_WORKLOAD = "v720x1280x129"

@@ -77,7 +77,8 @@ def test_full_output_parity(name):
     full_check(inp, wl.grid, wl.text_len)
 
 
-@pytest.mark.parametrize("name", ["v544x960x129", "v720x1280x129"])
+@pytest.mark.parametrize("name", ["v544x960x129", "v720x1280x129", "v960x960x129", "v1104x832x129",
+                                  "cfg544x960x129"])
 def test_sampled_parity_large(name):
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl, seed=2)
@@ -193,7 +194,8 @@ def _run_both(inp, grid, text_len, theta=256.0):
     return fused, two, ws
 
 
-@pytest.mark.parametrize("name", ["tiny", "img256", "v544x960x17", "v720x1280x129"])
+@pytest.mark.parametrize("name", ["tiny", "img256", "v544x960x17", "v720x1280x129", "v1104x832x129",
+                                  "cfg544x960x129"])
 def test_workspace_path_bit_identical(name):
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl, seed=4)
