@@ -47,8 +47,19 @@ constexpr int BM = 128;             // query rows per Q tile
 constexpr int BN = 128;             // keys per K/V tile
 constexpr int QTILES = 2;           // Q tiles per work unit
 constexpr int UNIT_ROWS = BM * QTILES;
-constexpr int KSTAGES = 2;
-constexpr int VSTAGES = 2;
+// K and V tiles share a pool of KV_SLOTS shared-memory tiles: K takes the
+// first kstages slots and V the next vstages (chosen per launch). When the
+// RoPE warps rotate K, three K stages and one V stage let them work on K tiles
+// up to two tiles ahead of the tensor core; pre-rotated keys need no lead and
+// keep two of each.
+constexpr int KV_SLOTS = 4;
+constexpr int KSTAGES_MAX = 3;
+constexpr int VSTAGES_MAX = 2;
+constexpr int KSTAGES_ROPE = 3, VSTAGES_ROPE = 1;
+constexpr int KSTAGES_ROTATED = 2, VSTAGES_ROTATED = 2;
+static_assert(KSTAGES_ROPE + VSTAGES_ROPE <= KV_SLOTS && KSTAGES_ROTATED + VSTAGES_ROTATED <= KV_SLOTS, "KV pool");
+static_assert(KSTAGES_ROPE <= KSTAGES_MAX && KSTAGES_ROTATED <= KSTAGES_MAX, "K stages");
+static_assert(VSTAGES_ROPE <= VSTAGES_MAX && VSTAGES_ROTATED <= VSTAGES_MAX, "V stages");
 constexpr int BOX_BYTES = 128 * 64 * 2;   // 128 rows x 64 channels bf16, 128B-swizzled
 constexpr int TILE_BYTES = 2 * BOX_BYTES; // 128 rows x 128 channels
 
@@ -72,21 +83,20 @@ static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL <= N
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + QTILES * TILE_BYTES;
-constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
+constexpr int OFF_KV = OFF_Q + QTILES * TILE_BYTES;
 // cos/sin table of the rotation angles: a cos and a sin per (axis, position,
 // pair) = 8*T + 28*(Hp + Wp) entries of 8 bytes, built once per CTA.
-constexpr int OFF_TABLE = OFF_V + VSTAGES * TILE_BYTES;
+constexpr int OFF_TABLE = OFF_KV + KV_SLOTS * TILE_BYTES;
 constexpr int TABLE_MAX_ENTRIES = 4096;
 constexpr int OFF_BAR = OFF_TABLE + TABLE_MAX_ENTRIES * 8;
 // barrier indices
 constexpr int B_Q_FULL = 0, B_Q_READY = 1, B_Q_EMPTY = 2;
 constexpr int B_K_FULL = 3;
-constexpr int B_K_READY = B_K_FULL + KSTAGES;
-constexpr int B_K_EMPTY = B_K_READY + KSTAGES;
-constexpr int B_V_FULL = B_K_EMPTY + KSTAGES;
-constexpr int B_V_EMPTY = B_V_FULL + VSTAGES;
-constexpr int B_S_FULL = B_V_EMPTY + VSTAGES;
+constexpr int B_K_READY = B_K_FULL + KSTAGES_MAX;
+constexpr int B_K_EMPTY = B_K_READY + KSTAGES_MAX;
+constexpr int B_V_FULL = B_K_EMPTY + KSTAGES_MAX;
+constexpr int B_V_EMPTY = B_V_FULL + VSTAGES_MAX;
+constexpr int B_S_FULL = B_V_EMPTY + VSTAGES_MAX;
 constexpr int B_P_READY = B_S_FULL + QTILES;
 constexpr int B_O_DONE = B_P_READY + QTILES;
 constexpr int B_DRAIN = B_O_DONE + QTILES;
@@ -116,6 +126,8 @@ struct __align__(64) Params {
     int B, H, S, N, T, Hp, Wp, HpWp;
     int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
     int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
+    int kstages;        // K tiles in flight (slots 0 .. kstages-1 of the KV pool)
+    int vstages;        // V tiles in flight (the next vstages slots)
     int n_qunits;       // ceil(S / 256)
     int units;          // B * H * n_qunits
     float theta_log2;   // log2(rope_theta)
@@ -153,6 +165,19 @@ struct Waiter {
         int ok = 1;
         if ((threadIdx.x & 31) == 0) ok = wait(bar, parity, role) ? 1 : 0;
         return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    }
+};
+
+// Position in a ring of n stages: the stage in use and the parity of its
+// current fill (flips each time the ring wraps).
+struct Ring {
+    uint32_t n, s, ph;
+    __device__ __forceinline__ explicit Ring(int stages) : n(static_cast<uint32_t>(stages)), s(0), ph(0) {}
+    __device__ __forceinline__ void next() {
+        if (++s == n) {
+            s = 0;
+            ph ^= 1u;
+        }
     }
 };
 
@@ -345,7 +370,8 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
     const RopeLane L = make_rope_lane(rt, p);
     const int lane = threadIdx.x & 31;
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-    uint32_t kt = 0, lu = 0;
+    Ring kr(p.kstages);
+    uint32_t lu = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
         const UnitCoord c = decode_unit(p, u);
         if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
@@ -355,13 +381,12 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         if (lane == 0) mbar_arrive(bar(B_Q_READY));
         bool ok = true;
         if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
-        for (int j = 0; j < c.nt; ++j, ++kt) {
-            const uint32_t sk = kt % KSTAGES;
-            if (!(ok = waiter.wait_warp(bar(B_K_FULL + sk), (kt / KSTAGES) & 1, ROLE_ROPE))) break;
-            if (j * BN < p.N) rope_tile(sK + sk * TILE_BYTES, sTable, j * BN, rt, L, p);
+        for (int j = 0; j < c.nt; ++j, kr.next()) {
+            if (!(ok = waiter.wait_warp(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
+            if (j * BN < p.N) rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_K_READY + sk));
+            if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
         }
         if (!ok) break;
     }
@@ -407,12 +432,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         mbar_init(bar(B_Q_FULL), 1);
         mbar_init(bar(B_Q_READY), ROPE_WARPS);
         mbar_init(bar(B_Q_EMPTY), 1);
-        for (int s = 0; s < KSTAGES; ++s) {
+        for (int s = 0; s < KSTAGES_MAX; ++s) {
             mbar_init(bar(B_K_FULL + s), 1);
             mbar_init(bar(B_K_READY + s), ROPE_WARPS);
             mbar_init(bar(B_K_EMPTY + s), 1);
         }
-        for (int s = 0; s < VSTAGES; ++s) {
+        for (int s = 0; s < VSTAGES_MAX; ++s) {
             mbar_init(bar(B_V_FULL + s), 1);
             mbar_init(bar(B_V_EMPTY + s), 1);
         }
@@ -437,8 +462,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
 
     const Waiter waiter{abort_flag, p.timeout_ns};
     const uint32_t sQ = base + OFF_Q;
-    const uint32_t sK = base + OFF_K;
-    const uint32_t sV = base + OFF_V;
+    const uint32_t sK = base + OFF_KV;
+    const uint32_t sV = sK + static_cast<uint32_t>(p.kstages) * TILE_BYTES;
     const uint32_t sTable = base + OFF_TABLE;
 
     if (warp >= WARP_TMA) {
@@ -449,39 +474,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             tma_prefetch_desc(&p.tm_q);
             tma_prefetch_desc(&p.tm_k);
             tma_prefetch_desc(&p.tm_v);
-            uint32_t kt = 0, vt = 0, lu = 0;
+            // Two cursors over this CTA's (unit, tile) sequence: keys (each
+            // unit's Q ahead of its first key) run up to kstages tiles ahead
+            // of the values.
+            Ring kr(p.kstages), vr(p.vstages);
+            uint32_t kt = 0, vt = 0, klu = 0;   // K and V tiles issued, units whose Q is issued
+            int ku = blockIdx.x, kj = 0, vu = blockIdx.x, vj = 0;
+            UnitCoord kc{}, vc{};
+            if (ku < p.units) kc = vc = decode_unit(p, ku);
             // stages with a load in flight and the parity it completes (bit per stage)
             uint32_t armed_q = 0, armed_k = 0, armed_v = 0;
             uint32_t par_q = 0, par_k = 0, par_v = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
-                const UnitCoord c = decode_unit(p, u);
-                if (!(ok = waiter.wait(bar(B_Q_EMPTY), (lu & 1) ^ 1, ROLE_TMA))) break;
-                mbar_arrive_expect_tx(bar(B_Q_FULL), QTILES * TILE_BYTES);
-                armed_q = 1; par_q = lu & 1;
-                for (int qi = 0; qi < QTILES; ++qi)
+            while (ok && vu < p.units) {
+                while (ku < p.units && kt < vt + kr.n) {
+                    if (kj == 0) {
+                        // The Q buffer frees when the previous unit's last QK
+                        // MMA completes, which needs that unit's values up to
+                        // its second-last tile: issue those before waiting.
+                        if (kt >= vt + 2) break;
+                        if (!(ok = waiter.wait(bar(B_Q_EMPTY), (klu & 1) ^ 1, ROLE_TMA))) break;
+                        mbar_arrive_expect_tx(bar(B_Q_FULL), QTILES * TILE_BYTES);
+                        armed_q = 1; par_q = klu & 1;
+                        for (int qi = 0; qi < QTILES; ++qi)
+                            for (int bx = 0; bx < 2; ++bx)
+                                tma_load_4d(sQ + qi * TILE_BYTES + bx * BOX_BYTES, &p.tm_q, bar(B_Q_FULL), bx * 64,
+                                            kc.h, kc.qu * UNIT_ROWS + qi * BM, kc.b);
+                    }
+                    if (!(ok = waiter.wait(bar(B_K_EMPTY + kr.s), kr.ph ^ 1, ROLE_TMA))) break;
+                    mbar_arrive_expect_tx(bar(B_K_FULL + kr.s), TILE_BYTES);
+                    armed_k |= 1u << kr.s;
+                    par_k = (par_k & ~(1u << kr.s)) | (kr.ph << kr.s);
                     for (int bx = 0; bx < 2; ++bx)
-                        tma_load_4d(sQ + qi * TILE_BYTES + bx * BOX_BYTES, &p.tm_q, bar(B_Q_FULL), bx * 64, c.h,
-                                    c.qu * UNIT_ROWS + qi * BM, c.b);
-                for (int j = 0; j < c.nt; ++j) {
-                    const uint32_t sk = kt % KSTAGES, pk = (kt / KSTAGES) & 1;
-                    if (!(ok = waiter.wait(bar(B_K_EMPTY + sk), pk ^ 1, ROLE_TMA))) break;
-                    mbar_arrive_expect_tx(bar(B_K_FULL + sk), TILE_BYTES);
-                    armed_k |= 1u << sk;
-                    par_k = (par_k & ~(1u << sk)) | (pk << sk);
-                    for (int bx = 0; bx < 2; ++bx)
-                        tma_load_4d(sK + sk * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + sk), bx * 64, c.h,
-                                    j * BN, c.b);
+                        tma_load_4d(sK + kr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + kr.s), bx * 64,
+                                    kc.h, kj * BN, kc.b);
+                    kr.next();
                     ++kt;
-                    const uint32_t sv = vt % VSTAGES, pv = (vt / VSTAGES) & 1;
-                    if (!(ok = waiter.wait(bar(B_V_EMPTY + sv), pv ^ 1, ROLE_TMA))) break;
-                    mbar_arrive_expect_tx(bar(B_V_FULL + sv), TILE_BYTES);
-                    armed_v |= 1u << sv;
-                    par_v = (par_v & ~(1u << sv)) | (pv << sv);
-                    for (int bx = 0; bx < 2; ++bx)
-                        tma_load_4d(sV + sv * TILE_BYTES + bx * BOX_BYTES, &p.tm_v, bar(B_V_FULL + sv), bx * 64, c.h,
-                                    j * BN, c.b);
-                    ++vt;
+                    if (++kj == kc.nt) {
+                        kj = 0;
+                        ++klu;
+                        ku += gridDim.x;
+                        if (ku < p.units) kc = decode_unit(p, ku);
+                    }
+                }
+                if (!ok) break;
+                if (!(ok = waiter.wait(bar(B_V_EMPTY + vr.s), vr.ph ^ 1, ROLE_TMA))) break;
+                mbar_arrive_expect_tx(bar(B_V_FULL + vr.s), TILE_BYTES);
+                armed_v |= 1u << vr.s;
+                par_v = (par_v & ~(1u << vr.s)) | (vr.ph << vr.s);
+                for (int bx = 0; bx < 2; ++bx)
+                    tma_load_4d(sV + vr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_v, bar(B_V_FULL + vr.s), bx * 64,
+                                vc.h, vj * BN, vc.b);
+                vr.next();
+                ++vt;
+                if (++vj == vc.nt) {
+                    vj = 0;
+                    vu += gridDim.x;
+                    if (vu < p.units) vc = decode_unit(p, vu);
                 }
             }
             if (!ok) {
@@ -490,9 +539,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 volatile int never = 0;
                 Waiter tail{&never, 20000000ull};
                 if (armed_q) tail.wait(bar(B_Q_FULL), par_q, ROLE_TMA);
-                for (int s = 0; s < KSTAGES; ++s)
+                for (int s = 0; s < p.kstages; ++s)
                     if ((armed_k >> s) & 1u) tail.wait(bar(B_K_FULL + s), (par_k >> s) & 1u, ROLE_TMA);
-                for (int s = 0; s < VSTAGES; ++s)
+                for (int s = 0; s < p.vstages; ++s)
                     if ((armed_v >> s) & 1u) tail.wait(bar(B_V_FULL + s), (par_v >> s) & 1u, ROLE_TMA);
             }
         }
@@ -505,26 +554,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             // K tiles are ready for the tensor core once the RoPE warps have
             // rotated them, or, when they arrive rotated, once TMA lands them.
             const int k_ready = p.k_rotated ? B_K_FULL : B_K_READY;
-            uint32_t kt = 0, vt = 0, lu = 0;
+            Ring kr(p.kstages), vr(p.vstages);
+            uint32_t lu = 0;
             uint32_t pr[QTILES] = {0, 0};
             bool ok = true;
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
                 const UnitCoord c = decode_unit(p, u);
                 if (!(ok = waiter.wait(bar(B_Q_READY), lu & 1, ROLE_MMA))) break;
-                uint32_t sk = kt % KSTAGES;
-                if (!(ok = waiter.wait(bar(k_ready + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                if (!(ok = waiter.wait(bar(k_ready + kr.s), kr.ph, ROLE_MMA))) break;
                 tc_fence_after();
-                issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
+                issue_qk(tmem_base + TM_S + 0, sQ, sK + kr.s * TILE_BYTES);
                 mma_commit(bar(B_S_FULL + 0));
-                issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + sk * TILE_BYTES);
+                issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + kr.s * TILE_BYTES);
                 mma_commit(bar(B_S_FULL + 1));
-                mma_commit(bar(B_K_EMPTY + sk));
-                ++kt;
+                mma_commit(bar(B_K_EMPTY + kr.s));
+                kr.next();
                 if (c.nt == 1) mma_commit(bar(B_Q_EMPTY));
                 for (int j = 0; j < c.nt; ++j) {
-                    const uint32_t sv = vt % VSTAGES;
-                    if (!(ok = waiter.wait(bar(B_V_FULL + sv), (vt / VSTAGES) & 1, ROLE_MMA))) break;
-                    const uint32_t v_tile = sV + sv * TILE_BYTES;
+                    if (!(ok = waiter.wait(bar(B_V_FULL + vr.s), vr.ph, ROLE_MMA))) break;
+                    const uint32_t v_tile = sV + vr.s * TILE_BYTES;
                     // Q tile 0: PV for tile j, then QK for tile j+1
                     if (!(ok = waiter.wait(bar(B_P_READY + 0), pr[0] & 1, ROLE_MMA))) break;
                     ++pr[0];
@@ -532,11 +580,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     issue_pv(tmem_base + TM_O + 0, tmem_base + TM_S + 0, v_tile, j > 0);
                     if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 0));
                     const bool more = j + 1 < c.nt;
-                    sk = kt % KSTAGES;
+                    const uint32_t k_tile = sK + kr.s * TILE_BYTES;
                     if (more) {
-                        if (!(ok = waiter.wait(bar(k_ready + sk), (kt / KSTAGES) & 1, ROLE_MMA))) break;
+                        if (!(ok = waiter.wait(bar(k_ready + kr.s), kr.ph, ROLE_MMA))) break;
                         tc_fence_after();
-                        issue_qk(tmem_base + TM_S + 0, sQ, sK + sk * TILE_BYTES);
+                        issue_qk(tmem_base + TM_S + 0, sQ, k_tile);
                         mma_commit(bar(B_S_FULL + 0));
                     }
                     // Q tile 1
@@ -544,14 +592,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     ++pr[1];
                     tc_fence_after();
                     issue_pv(tmem_base + TM_O + 128, tmem_base + TM_S + 128, v_tile, j > 0);
-                    mma_commit(bar(B_V_EMPTY + sv));
-                    ++vt;
+                    mma_commit(bar(B_V_EMPTY + vr.s));
+                    vr.next();
                     if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 1));
                     if (more) {
-                        issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + sk * TILE_BYTES);
+                        issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, k_tile);
                         mma_commit(bar(B_S_FULL + 1));
-                        mma_commit(bar(B_K_EMPTY + sk));
-                        ++kt;
+                        mma_commit(bar(B_K_EMPTY + kr.s));
+                        kr.next();
                         if (j + 1 == c.nt - 1) mma_commit(bar(B_Q_EMPTY));
                     }
                 }
@@ -896,6 +944,8 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->Wp = Wp;
     prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
     prm->k_rotated = k_rotated ? 1 : 0;
+    prm->kstages = k_rotated ? KSTAGES_ROTATED : KSTAGES_ROPE;
+    prm->vstages = k_rotated ? VSTAGES_ROTATED : VSTAGES_ROPE;
     prm->HpWp = Hp * Wp;
     prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
     prm->units = static_cast<int>(call.units);
