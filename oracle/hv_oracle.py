@@ -19,6 +19,8 @@ Sources (pages on HunyuanVideo; cited by page title and section):
     -> 33x45x80 = 118800.
   - §5.2 "双流块": Q=[Q_v;Q_t] (same for K, V), Attn = softmax(QK^T/sqrt(128))V,
     joint length S = N + L with L the valid text length.
+  - §5.4 "归一化、条件调制和残差门": RMSNorm on the Q and K of every
+    attention head, RMSNorm(x) = gamma * x / sqrt((1/d) sum_j x_j^2 + eps).
   - §5.5 "3D RoPE": q'_p = R(p) q_p, k'_p = R(p) k_p; head dim 128 split
     (d_t, d_h, d_w) = (16, 56, 56); R_3D = R_t (+) R_h (+) R_w; theta = 256;
     applied to the video Q, K only, text tokens are not rotated.
@@ -49,6 +51,15 @@ Readings where the pages are silent (each also listed in the design doc):
      N + valid are masked out; padded text *query* rows are computed like any
      other row (they attend to the valid keys).
   R8 scale is a parameter, default 1/sqrt(128).
+  R13 QK RMSNorm ([P1] §5.4, optional prologue): over the head dim d = 128 of
+     each (token, head) row, y = gamma * x / sqrt(mean_j x_j^2 + eps), with one
+     gamma of 128 channels shared by all heads (the formula has no head index).
+  R14 video rows take the video stream's gamma, text rows the text stream's
+     ([P1] §5.2: the double-stream blocks keep separate parameters per
+     modality); a single-stream block passes the same gamma twice.
+  R15 order: RMSNorm first, then the 3D rotation of the video rows (the norm
+     acts on Q, K as projected, §5.4; RoPE rotates the Q, K that attention
+     uses, §5.5). eps is a parameter (the pages give none).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, invariants, a second independent formulation, a library SDPA
@@ -163,9 +174,33 @@ def rotate_sequence(x: np.ndarray, grid: tuple[int, int, int], theta: float = DE
     return out
 
 
+def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis ([P1] §5.4): gamma * x / sqrt(mean(x^2) + eps).
+
+    x: (..., d) float64; gamma: (d,). Returns a new float64 array.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    gamma = np.asarray(gamma, dtype=np.float64)
+    assert gamma.shape == (x.shape[-1],)
+    mean_sq = np.mean(x * x, axis=-1, keepdims=True)
+    return gamma * (x / np.sqrt(mean_sq + eps))
+
+
+def qk_norm_rows(x: np.ndarray, is_video: np.ndarray, gamma_video: np.ndarray, gamma_text: np.ndarray,
+                 eps: float) -> np.ndarray:
+    """Per-head QK RMSNorm of rows of one head (R13-R14): video rows with the
+    video stream's gamma, text rows with the text stream's gamma."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    vid = np.asarray(is_video, dtype=bool)
+    out[vid] = rms_norm(x[vid], gamma_video, eps)
+    out[~vid] = rms_norm(x[~vid], gamma_text, eps)
+    return out
+
+
 def joint_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tuple[int, int, int],
                          valid: int, theta: float = DEFAULT_THETA, scale: float | None = None,
-                         rows: np.ndarray | None = None) -> np.ndarray:
+                         rows: np.ndarray | None = None, qk_norm: dict | None = None) -> np.ndarray:
     """Joint full attention of one (batch, head), float64.
 
     [P1] §5.2: over the concatenation [video ; text] compute
@@ -173,7 +208,9 @@ def joint_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tupl
     (§5.5, video rows only). Keys are the N video tokens and the first
     ``valid`` text tokens (joint length N + L, L the valid text length);
     padded keys take no part (R7). ``rows`` selects query rows (default: all
-    S rows, padded text rows included).
+    S rows, padded text rows included). ``qk_norm``, if given, is a dict with
+    gamma_q_video, gamma_k_video, gamma_q_text, gamma_k_text (128 each) and
+    eps: the RMSNorm prologue (R13-R15), applied before the rotation.
 
     q, k, v: (S, 128). Returns (len(rows), 128) float64.
     """
@@ -190,10 +227,15 @@ def joint_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tupl
     kv_len = n + valid
 
     qr = np.asarray(q, dtype=np.float64)[rows].copy()
+    kr = np.asarray(k, dtype=np.float64)[:kv_len].copy()
     vid = rows < n
+    if qk_norm is not None:
+        eps = float(qk_norm["eps"])
+        qr = qk_norm_rows(qr, vid, qk_norm["gamma_q_video"], qk_norm["gamma_q_text"], eps)
+        kr = qk_norm_rows(kr, np.arange(kv_len) < n, qk_norm["gamma_k_video"], qk_norm["gamma_k_text"], eps)
     if vid.any():
         qr[vid] = rope3d_rotate(qr[vid], token_positions(t_lat, hp, wp)[rows[vid]], theta)
-    kr = rotate_sequence(np.asarray(k, dtype=np.float64)[:kv_len], grid, theta)
+    kr = rotate_sequence(kr, grid, theta)
     vv = np.asarray(v, dtype=np.float64)[:kv_len]
 
     scores = (qr @ kr.T) * scale                     # (rows, N + valid)
@@ -205,7 +247,7 @@ def joint_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tupl
 
 def joint_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tuple[int, int, int],
                     text_len: int, text_valid, theta: float = DEFAULT_THETA,
-                    scale: float | None = None) -> np.ndarray:
+                    scale: float | None = None, qk_norm: dict | None = None) -> np.ndarray:
     """Full output [B, S, heads, 128] float64 of the joint attention call.
 
     Inputs in the boundary layout [B, S, heads, 128] with S = N + text_len
@@ -218,13 +260,13 @@ def joint_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tuple[int
     for b in range(b_sz):
         for h in range(heads):
             out[b, :, h, :] = joint_attention_head(q[b, :, h], k[b, :, h], v[b, :, h], grid,
-                                                   int(text_valid[b]), theta, scale)
+                                                   int(text_valid[b]), theta, scale, qk_norm=qk_norm)
     return out
 
 
 def joint_attention_samples(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tuple[int, int, int],
                             text_len: int, text_valid, samples: np.ndarray, theta: float = DEFAULT_THETA,
-                            scale: float | None = None) -> np.ndarray:
+                            scale: float | None = None, qk_norm: dict | None = None) -> np.ndarray:
     """Outputs of selected (b, head, row) triples, float64, shape (n_samples, 128).
 
     Same definition as ``joint_attention``; heads are grouped so that each
@@ -237,7 +279,7 @@ def joint_attention_samples(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: t
         sel = np.nonzero(keys == key)[0]
         b, h = int(samples[sel[0], 0]), int(samples[sel[0], 1])
         out[sel] = joint_attention_head(q[b, :, h], k[b, :, h], v[b, :, h], grid,
-                                        int(text_valid[b]), theta, scale, rows=samples[sel, 2])
+                                        int(text_valid[b]), theta, scale, rows=samples[sel, 2], qk_norm=qk_norm)
     return out
 
 
