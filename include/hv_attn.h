@@ -40,8 +40,8 @@ enum hv_status {
     HV_ERR_BAD_SHAPE = 3,      /* B, heads, T, Hp or Wp < 1, or B > HV_MAX_BATCH     */
     HV_ERR_BAD_TEXT = 4,       /* text_len not in [0,256] or text_valid[b] not in [0,text_len] */
     HV_ERR_TOO_LARGE = 5,      /* S*heads*128 or a TMA coordinate exceeds int32      */
-    HV_ERR_ALIAS = 6,          /* out overlaps q, k or v                             */
-    HV_ERR_BAD_SCALAR = 7,     /* rope_theta <= 0 or not finite, scale not finite    */
+    HV_ERR_ALIAS = 6,          /* out overlaps q, k, v (or qk_gamma)                 */
+    HV_ERR_BAD_SCALAR = 7,     /* rope_theta <= 0 or not finite, scale not finite, qk_eps < 0 or not finite */
     HV_ERR_NO_DEVICE = 8,      /* current CUDA device is not an sm_100 (B200) part   */
     HV_ERR_LAUNCH = 9,         /* a CUDA runtime/driver call failed                  */
     HV_ERR_DEVICE_TIMEOUT = 10,/* a kernel-side wait ran out (see hv_attn_last_device_error) */
@@ -110,6 +110,49 @@ int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out,
                        int text_len, const int* text_valid,
                        float rope_theta, float scale,
                        void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * hv_attn_forward_qknorm - hv_attn_forward with the per-head QK RMSNorm
+ * prologue of the DiT blocks (§5.4 "归一化、条件调制和残差门": RMSNorm on the Q
+ * and K of every attention head): before the rotation, every Q and K row
+ * (one token, one head, 128 channels) becomes
+ *   y = gamma * x / sqrt((1/128) sum_j x_j^2 + eps),
+ * video rows with the video stream's gamma and text rows with the text
+ * stream's (the double-stream blocks keep separate parameters per modality,
+ * §5.2; a single-stream block passes the same gamma twice). Then video rows
+ * are rotated as in hv_attn_forward and attention is computed on the result.
+ * The normalised, rotated rows are rounded to bf16 once, as the rotation
+ * alone is.
+ *
+ * qk_gamma : DEVICE pointer, fp32 [4][128], 16-byte aligned, owned by the
+ *            caller: gamma of Q video rows, K video rows, Q text rows, K text
+ *            rows, in that order; shared by all heads. Must not overlap out.
+ * qk_eps   : epsilon inside the root (finite, >= 0; the pages give no value,
+ *            1e-6 is usual).
+ * Other arguments, ownership, asynchrony and errors as hv_attn_forward;
+ * HV_ERR_NULL_POINTER / HV_ERR_MISALIGNED / HV_ERR_BAD_SCALAR / HV_ERR_ALIAS
+ * also cover qk_gamma and qk_eps.
+ */
+int hv_attn_forward_qknorm(const void* q, const void* k, const void* v, void* out,
+                           int B, int heads, int T, int Hp, int Wp,
+                           int text_len, const int* text_valid,
+                           float rope_theta, float scale,
+                           const float* qk_gamma, float qk_eps, void* cuda_stream);
+
+/*
+ * hv_attn_forward_qknorm_ws - hv_attn_forward_qknorm in the two stages of
+ * hv_attn_forward_ws: the first kernel writes the normalised, rotated keys
+ * into `workspace` (text rows normalised), the attention kernel normalises
+ * and rotates Q on load. Output bit-identical to hv_attn_forward_qknorm.
+ * Arguments as hv_attn_forward_qknorm plus workspace / workspace_bytes as in
+ * hv_attn_forward_ws (the workspace must not overlap qk_gamma either).
+ */
+int hv_attn_forward_qknorm_ws(const void* q, const void* k, const void* v, void* out,
+                              int B, int heads, int T, int Hp, int Wp,
+                              int text_len, const int* text_valid,
+                              float rope_theta, float scale,
+                              const float* qk_gamma, float qk_eps,
+                              void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
  * hv_attn_workspace_bytes - workspace hv_attn_forward_ws needs:

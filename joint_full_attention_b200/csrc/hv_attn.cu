@@ -87,8 +87,14 @@ constexpr int OFF_KV = OFF_Q + QTILES * TILE_BYTES;
 // cos/sin table of the rotation angles: a cos and a sin per (axis, position,
 // pair) = 8*T + 28*(Hp + Wp) entries of 8 bytes, built once per CTA.
 constexpr int OFF_TABLE = OFF_KV + KV_SLOTS * TILE_BYTES;
-constexpr int TABLE_MAX_ENTRIES = 4096;
-constexpr int OFF_BAR = OFF_TABLE + TABLE_MAX_ENTRIES * 8;
+// 3840 entries cover every size of the pages' supported-size table (720p
+// needs 3764); larger grids compute (cos, sin) per pair instead.
+constexpr int TABLE_MAX_ENTRIES = 3840;
+// QK RMSNorm gammas (fp32 [4][128]: Q video, K video, Q text, K text), copied
+// in at kernel start when the prologue is on.
+constexpr int OFF_GAMMA = OFF_TABLE + TABLE_MAX_ENTRIES * 8;
+constexpr int GAMMA_BYTES = 4 * D * 4;
+constexpr int OFF_BAR = OFF_GAMMA + GAMMA_BYTES;
 // barrier indices
 constexpr int B_Q_FULL = 0, B_Q_READY = 1, B_Q_EMPTY = 2;
 constexpr int B_K_FULL = 3;
@@ -126,6 +132,9 @@ struct __align__(64) Params {
     int B, H, S, N, T, Hp, Wp, HpWp;
     int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
     int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
+    int qk_norm;        // 1: RMSNorm the Q and K rows (gammas below) before rotating them
+    float qk_eps;       // RMSNorm epsilon
+    const float* qk_gamma;   // device, fp32 [4][128]: Q video, K video, Q text, K text
     int kstages;        // K tiles in flight (slots 0 .. kstages-1 of the KV pool)
     int vstages;        // V tiles in flight (the next vstages slots)
     int n_qunits;       // ceil(S / 256)
@@ -204,6 +213,7 @@ __device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
 // Axis t: channels [0,16), 8 pairs; h: [16,72), 28 pairs; w: [72,128), 28 pairs.
 struct RopeLane {
     int box, cin, axis;
+    int ch0;           // first of the chunk's 8 channels
     int i0;            // first pair index of the chunk inside its axis segment
     int half_dim;      // pairs in the axis segment (8 or 28)
     int table_base;    // first table float of the axis segment
@@ -229,6 +239,7 @@ __device__ __forceinline__ RopeLane make_rope_lane(int rt, const Params& p) {
     L.box = cc >> 3;
     L.cin = cc & 7;
     const int ch0 = cc * 8;
+    L.ch0 = ch0;
     int dax;
     if (ch0 < 16) {
         L.axis = 0; L.i0 = ch0 / 2; dax = 16; L.table_base = 0;
@@ -266,12 +277,40 @@ __device__ __forceinline__ void build_rope_table(float* table, const Params& p) 
 
 // Explicitly rounded operations (no contraction choices left to the
 // compiler), so that every kernel rotating a pair gets the same bits.
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
-    const float x0 = __uint_as_float(w << 16);          // channel 2i   (low half)
-    const float x1 = __uint_as_float(w & 0xFFFF0000u);  // channel 2i+1 (high half)
+__device__ __forceinline__ uint32_t rotate_f(float x0, float x1, float cs, float sn) {
     const float y0 = __fmaf_rn(x0, cs, -__fmul_rn(x1, sn));
     const float y1 = __fmaf_rn(x0, sn, __fmul_rn(x1, cs));
     return pack_bf16x2(y0, y1);
+}
+
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
+    // channel 2i in the low half, 2i+1 in the high half
+    return rotate_f(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u), cs, sn);
+}
+
+// QK RMSNorm of one row ("HunyuanVideo 模型结构与数学原理" §5.4):
+// y = gamma * x / sqrt(mean_j x_j^2 + eps) over the 128 channels. The row's 16
+// chunks of 8 channels sit in the 16 lanes of one half-warp (lane & 15 =
+// chunk); every lane of the warp must call this together. The sum of squares
+// is taken in a fixed order (channel order, then a butterfly over the half-
+// warp), so every kernel that normalises a row this way gets the same bits.
+__device__ __forceinline__ void rms_norm_chunk(uint4 d, float4 g0, float4 g1, float eps, float (&y)[8]) {
+    const uint32_t w[4] = {d.x, d.y, d.z, d.w};
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        x[2 * q] = __uint_as_float(w[q] << 16);
+        x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+    float ss = __fmul_rn(x[0], x[0]);
+#pragma unroll
+    for (int c = 1; c < 8; ++c) ss = __fmaf_rn(x[c], x[c], ss);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    const float r = rsqrtf(__fmaf_rn(ss, 1.f / D, eps));
+    const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[c] = __fmul_rn(__fmul_rn(x[c], r), g[c]);
 }
 
 
@@ -363,10 +402,78 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
     }
 }
 
+// RMSNorm prologue, then the rotation of the video rows, for every row of a
+// tile (rows rb, rb + 12, ...); text rows and rows past the sequence are only
+// normalised (rows past the sequence hold TMA's zero fill and stay zero).
+// gamma_v / gamma_t: shared-memory addresses of the video / text gamma of
+// this tensor (Q or K). Every lane of a warp runs the same number of
+// iterations (rb and rb + 1 share a warp and a trip count), as the row sum is
+// a half-warp shuffle.
+__device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
+                                               int n0, int rt, const RopeLane& L, const Params& p) {
+    const int rb = rt >> 4;
+    int n = n0 + rb;
+    GridPos g;
+    g.w = n % p.Wp;
+    const int th = n / p.Wp;
+    g.h = th % p.Hp;
+    g.t = th / p.Hp;
+    const uint32_t box_base = tile + L.box * BOX_BYTES;
+    const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
+    const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
+    const int stride = 2 * L.half_dim;
+    const uint32_t gofs = 4u * static_cast<uint32_t>(L.ch0);
+#pragma unroll 1
+    for (int r = rb; r < BM; r += ROPE_GROUPS) {
+        const bool video = n < p.N;
+        const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
+        const uint32_t a = box_base + r * 128 + ((L.cin ^ (r & 7)) << 4);
+        const uint4 d = lds128(a);
+        const uint32_t gb = (video ? gamma_v : gamma_t) + gofs;
+        const uint4 g0 = lds128(gb), g1 = lds128(gb + 16);
+        uint4 c = make_uint4(0u, 0u, 0u, 0u), sn = c;
+        if (video && p.use_table) {
+            const uint32_t t = tab + 4u * static_cast<uint32_t>(pos * stride);
+            c = lds128(t);
+            sn = lds128(t + sin_off);
+        }
+        float y[8];
+        rms_norm_chunk(d, make_float4(__uint_as_float(g0.x), __uint_as_float(g0.y), __uint_as_float(g0.z),
+                                      __uint_as_float(g0.w)),
+                       make_float4(__uint_as_float(g1.x), __uint_as_float(g1.y), __uint_as_float(g1.z),
+                                   __uint_as_float(g1.w)),
+                       p.qk_eps, y);
+        uint32_t w[4];
+        if (video) {
+            if (p.use_table) {
+                const float cs[4] = {__uint_as_float(c.x), __uint_as_float(c.y), __uint_as_float(c.z),
+                                     __uint_as_float(c.w)};
+                const float ss[4] = {__uint_as_float(sn.x), __uint_as_float(sn.y), __uint_as_float(sn.z),
+                                     __uint_as_float(sn.w)};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) w[q] = rotate_f(y[2 * q], y[2 * q + 1], cs[q], ss[q]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float s1, c1;
+                    sincospif(angle_over_pi(pos, L.i0 + q, 2 * L.half_dim, p.theta_log2), &s1, &c1);
+                    w[q] = rotate_f(y[2 * q], y[2 * q + 1], c1, s1);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = pack_bf16x2(y[2 * q], y[2 * q + 1]);
+        }
+        sts128(a, make_uint4(w[0], w[1], w[2], w[3]));
+        n += ROPE_GROUPS;
+        advance8(g, p);
+    }
+}
+
 // The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
 // each to the MMA warp.
 __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
-                                          uint32_t sK, uint32_t sTable) {
+                                          uint32_t sK, uint32_t sTable, uint32_t sGamma) {
     const RopeLane L = make_rope_lane(rt, p);
     const int lane = threadIdx.x & 31;
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -375,7 +482,13 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
         const UnitCoord c = decode_unit(p, u);
         if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
-        for (int qi = 0; qi < QTILES; ++qi) rope_tile(sQ + qi * TILE_BYTES, sTable, c.qu * UNIT_ROWS + qi * BM, rt, L, p);
+        for (int qi = 0; qi < QTILES; ++qi) {
+            const int n0 = c.qu * UNIT_ROWS + qi * BM;
+            if (p.qk_norm)
+                rope_norm_tile(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, rt, L, p);
+            else
+                rope_tile(sQ + qi * TILE_BYTES, sTable, n0, rt, L, p);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_Q_READY));
@@ -383,7 +496,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
         for (int j = 0; j < c.nt; ++j, kr.next()) {
             if (!(ok = waiter.wait_warp(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
-            if (j * BN < p.N) rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, rt, L, p);
+            if (p.qk_norm)
+                rope_norm_tile(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, j * BN, rt, L, p);
+            else if (j * BN < p.N)
+                rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
@@ -455,6 +571,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         tmem_relinquish();
     }
     if (p.use_table) build_rope_table(reinterpret_cast<float*>(base_ptr + OFF_TABLE), p);
+    if (p.qk_norm) {
+        float* gdst = reinterpret_cast<float*>(base_ptr + OFF_GAMMA);
+        for (int i = threadIdx.x; i < 4 * D; i += blockDim.x) gdst[i] = __ldg(p.qk_gamma + i);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -465,6 +585,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     const uint32_t sK = base + OFF_KV;
     const uint32_t sV = sK + static_cast<uint32_t>(p.kstages) * TILE_BYTES;
     const uint32_t sTable = base + OFF_TABLE;
+    const uint32_t sGamma = base + OFF_GAMMA;
 
     if (warp >= WARP_TMA) {
       regs_decrease<REGS_CONTROL>();
@@ -547,7 +668,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
       } else if (warp > WARP_MMA) {
         // RoPE helpers: threads 128..191 of the RoPE role
-        rope_role(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable);
+        rope_role(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
@@ -616,7 +737,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     } else if (warp >= WARP_ROPE) {
         regs_decrease<REGS_ROPE>();
         // ------------------------------------------------------------ RoPE
-        rope_role(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable);
+        rope_role(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -743,26 +864,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
 // (four adjacent channel pairs of one axis segment); the same fp32 rotation
 // and bf16 rounding as the attention kernel's in-shared-memory path, with
 // (cos, sin) from sincospif of the same angles, so both paths agree bit for
-// bit. Memory-bound: reads and writes B*S*heads*256 bytes once.
+// bit. With the QK RMSNorm prologue (gamma_kv / gamma_kt non-null) every row
+// is first normalised as the attention kernel normalises it, and text rows
+// are normalised instead of copied. Memory-bound: reads and writes
+// B*S*heads*256 bytes once. Warps step through whole pairs of rows (16
+// chunks each), so a row's chunks always share a half-warp.
 __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict__ kin, uint4* __restrict__ kout,
                                                         long long n_chunks, int H, int S, int N, int Hp, int Wp,
-                                                        float theta_log2) {
+                                                        float theta_log2, const float* __restrict__ gamma_kv,
+                                                        const float* __restrict__ gamma_kt, float eps) {
     const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
-    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_chunks; e += step) {
-        uint4 d = __ldg(kin + e);
-        const int cc = static_cast<int>(e & 15);
+    const int lane = threadIdx.x & 31;
+    const bool norm = gamma_kv != nullptr;
+    for (long long e0 = static_cast<long long>(blockIdx.x) * blockDim.x + (threadIdx.x - lane); e0 < n_chunks;
+         e0 += step) {
+        const long long e = e0 + lane;
+        const bool live = e < n_chunks;
+        uint4 d = live ? __ldg(kin + e) : make_uint4(0u, 0u, 0u, 0u);
+        const int cc = lane & 15;
         const long long row = e >> 4;               // (b * S + s) * H + h
         const int s_idx = static_cast<int>((row / H) % S);
-        if (s_idx < N) {
-            const int ch0 = cc * 8;
-            int i0, dax, pos;
-            if (ch0 < 16) {
-                i0 = ch0 / 2; dax = 16; pos = s_idx / (Hp * Wp);
-            } else if (ch0 < 72) {
-                i0 = (ch0 - 16) / 2; dax = 56; pos = (s_idx / Wp) % Hp;
-            } else {
-                i0 = (ch0 - 72) / 2; dax = 56; pos = s_idx % Wp;
+        const bool video = s_idx < N;
+        const int ch0 = cc * 8;
+        int i0, dax, pos;
+        if (ch0 < 16) {
+            i0 = ch0 / 2; dax = 16; pos = s_idx / (Hp * Wp);
+        } else if (ch0 < 72) {
+            i0 = (ch0 - 16) / 2; dax = 56; pos = (s_idx / Wp) % Hp;
+        } else {
+            i0 = (ch0 - 72) / 2; dax = 56; pos = s_idx % Wp;
+        }
+        if (norm) {
+            const float* gsrc = (video ? gamma_kv : gamma_kt) + ch0;
+            float y[8];
+            rms_norm_chunk(d, __ldg(reinterpret_cast<const float4*>(gsrc)),
+                           __ldg(reinterpret_cast<const float4*>(gsrc + 4)), eps, y);
+            uint32_t wv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (video) {
+                    float sn, cs;
+                    sincospif(angle_over_pi(pos, i0 + q, dax, theta_log2), &sn, &cs);
+                    wv[q] = rotate_f(y[2 * q], y[2 * q + 1], cs, sn);
+                } else {
+                    wv[q] = pack_bf16x2(y[2 * q], y[2 * q + 1]);
+                }
             }
+            d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        } else if (video) {
             uint32_t wv[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -772,12 +921,10 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
             }
             d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        kout[e] = d;
+        if (live) kout[e] = d;
     }
 }
 
-// One warp waits on an mbarrier that nothing completes; the bounded wait must
-// run out, record ROLE_SELFTEST and return.
 __global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns) {
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int abort_flag;
@@ -863,6 +1010,12 @@ static bool overlaps(const void* a, const void* b, size_t bytes) {
     return x < y + bytes && y < x + bytes;
 }
 
+// [a, a + a_bytes) and [b, b + b_bytes) share a byte
+static bool ranges_overlap(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + b_bytes && y < x + a_bytes;
+}
+
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 
 struct Call {
@@ -871,8 +1024,21 @@ struct Call {
     size_t bytes = 0;   // bytes of one [B, S, heads, 128] bf16 tensor
 };
 
+// Checks of the QK RMSNorm arguments: gamma (device, fp32 [4][128], 16-byte
+// aligned, not overlapping out) and eps (finite, >= 0).
+static int validate_qk_norm(const float* qk_gamma, float eps, const void* out, size_t out_bytes) {
+    if (!qk_gamma) return HV_ERR_NULL_POINTER;
+    if (reinterpret_cast<uintptr_t>(qk_gamma) & 15u) return HV_ERR_MISALIGNED;
+    if (!std::isfinite(eps) || eps < 0.f) return HV_ERR_BAD_SCALAR;
+    if (ranges_overlap(out, out_bytes, qk_gamma, GAMMA_BYTES)) return HV_ERR_ALIAS;
+    return HV_OK;
+}
+
+// Argument checks (then the device): every error a call can report before
+// launching. qk_norm: also check the RMSNorm arguments qk_gamma / qk_eps.
 static int validate(const void* q, const void* k, const void* v, const void* out, int B, int heads, int T, int Hp,
-                    int Wp, int text_len, const int* text_valid, float rope_theta, float scale, Call& call) {
+                    int Wp, int text_len, const int* text_valid, float rope_theta, float scale, Call& call,
+                    bool qk_norm = false, const float* qk_gamma = nullptr, float qk_eps = 0.f) {
     if (!q || !k || !v || !out || !text_valid) return HV_ERR_NULL_POINTER;
     const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
@@ -889,6 +1055,10 @@ static int validate(const void* q, const void* k, const void* v, const void* out
         return HV_ERR_TOO_LARGE;
     const size_t bytes = static_cast<size_t>(B) * s_len * heads * D * 2;
     if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return HV_ERR_ALIAS;
+    if (qk_norm) {
+        const int st = validate_qk_norm(qk_gamma, qk_eps, out, bytes);
+        if (st != HV_OK) return st;
+    }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
     DeviceInfo& di = device_info(dev);
@@ -924,7 +1094,8 @@ static void* noalloc_scratch(int dev) {
 
 static int launch_attention(const Call& call, const void* q, const void* k, const void* v, void* out, int B,
                             int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
-                            float scale, bool k_rotated, cudaStream_t stream) {
+                            float scale, bool k_rotated, const float* qk_gamma, float qk_eps,
+                            cudaStream_t stream) {
     (void)text_len;
     Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
     std::memset(prm, 0, sizeof(Params));
@@ -944,6 +1115,9 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->Wp = Wp;
     prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
     prm->k_rotated = k_rotated ? 1 : 0;
+    prm->qk_norm = qk_gamma != nullptr ? 1 : 0;
+    prm->qk_eps = qk_eps;
+    prm->qk_gamma = qk_gamma;
     prm->kstages = k_rotated ? KSTAGES_ROTATED : KSTAGES_ROPE;
     prm->vstages = k_rotated ? VSTAGES_ROTATED : VSTAGES_ROPE;
     prm->HpWp = Hp * Wp;
@@ -958,6 +1132,18 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     delete prm;
     const cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
+}
+
+// First stage of the workspace paths: K' (rotated, and normalised when
+// qk_gamma is set) into `dst`.
+static int launch_rope_k(const Call& call, const void* k, void* dst, int heads, int Hp, int Wp, float rope_theta,
+                         const float* qk_gamma, float qk_eps, cudaStream_t stream) {
+    const long long n_chunks = static_cast<long long>(call.bytes / 16);
+    hv_rope_k_kernel<<<8 * call.sms, 256, 0, stream>>>(
+        static_cast<const uint4*>(k), static_cast<uint4*>(dst), n_chunks, heads, call.S, call.N, Hp, Wp,
+        static_cast<float>(std::log2(static_cast<double>(rope_theta))), qk_gamma ? qk_gamma + D : nullptr,
+        qk_gamma ? qk_gamma + 3 * D : nullptr, qk_eps);
+    return cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
 }  // namespace hv
@@ -998,7 +1184,19 @@ int hv_attn_forward(const void* q, const void* k, const void* v, void* out, int 
     int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call);
     if (st != HV_OK) return st;
     return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false,
-                            static_cast<cudaStream_t>(cuda_stream));
+                            nullptr, 0.f, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int hv_attn_forward_qknorm(const void* q, const void* k, const void* v, void* out, int B, int heads, int T, int Hp,
+                           int Wp, int text_len, const int* text_valid, float rope_theta, float scale,
+                           const float* qk_gamma, float qk_eps, void* cuda_stream) {
+    using namespace hv;
+    Call call;
+    int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call, true,
+                      qk_gamma, qk_eps);
+    if (st != HV_OK) return st;
+    return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false,
+                            qk_gamma, qk_eps, static_cast<cudaStream_t>(cuda_stream));
 }
 
 long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len) {
@@ -1019,14 +1217,30 @@ int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out, i
         overlaps(workspace, out, call.bytes))
         return HV_ERR_WORKSPACE;
     const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    const long long n_chunks = static_cast<long long>(call.bytes / 16);
-    const int grid = 8 * call.sms;
-    hv_rope_k_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<uint4*>(workspace), n_chunks,
-                                               heads, call.S, call.N, Hp, Wp,
-                                               static_cast<float>(std::log2(static_cast<double>(rope_theta))));
-    if (cudaGetLastError() != cudaSuccess) return HV_ERR_LAUNCH;
+    st = launch_rope_k(call, k, workspace, heads, Hp, Wp, rope_theta, nullptr, 0.f, stream);
+    if (st != HV_OK) return st;
     return launch_attention(call, q, workspace, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
-                            true, stream);
+                            true, nullptr, 0.f, stream);
+}
+
+int hv_attn_forward_qknorm_ws(const void* q, const void* k, const void* v, void* out, int B, int heads, int T,
+                              int Hp, int Wp, int text_len, const int* text_valid, float rope_theta, float scale,
+                              const float* qk_gamma, float qk_eps, void* workspace, size_t workspace_bytes,
+                              void* cuda_stream) {
+    using namespace hv;
+    Call call;
+    int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call, true,
+                      qk_gamma, qk_eps);
+    if (st != HV_OK) return st;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) || workspace_bytes < call.bytes ||
+        overlaps(workspace, q, call.bytes) || overlaps(workspace, k, call.bytes) || overlaps(workspace, v, call.bytes) ||
+        overlaps(workspace, out, call.bytes) || ranges_overlap(workspace, call.bytes, qk_gamma, GAMMA_BYTES))
+        return HV_ERR_WORKSPACE;
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    st = launch_rope_k(call, k, workspace, heads, Hp, Wp, rope_theta, qk_gamma, qk_eps, stream);
+    if (st != HV_OK) return st;
+    return launch_attention(call, q, workspace, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
+                            true, qk_gamma, qk_eps, stream);
 }
 
 int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int heads, int T,
@@ -1044,13 +1258,10 @@ int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* o
     // the first stage overwrites every byte of the scratch it uses, so
     // nothing left there by an earlier call needs clearing
     const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    const long long n_chunks = static_cast<long long>(call.bytes / 16);
-    hv_rope_k_kernel<<<8 * call.sms, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<uint4*>(scratch),
-                                                       n_chunks, heads, call.S, call.N, Hp, Wp,
-                                                       static_cast<float>(std::log2(static_cast<double>(rope_theta))));
-    if (cudaGetLastError() != cudaSuccess) return HV_ERR_LAUNCH;
+    st = launch_rope_k(call, k, scratch, heads, Hp, Wp, rope_theta, nullptr, 0.f, stream);
+    if (st != HV_OK) return st;
     return launch_attention(call, q, scratch, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
-                            true, stream);
+                            true, nullptr, 0.f, stream);
 }
 
 int hv_attn_last_device_error(void) {

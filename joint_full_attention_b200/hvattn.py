@@ -24,7 +24,8 @@ STATUS_NAMES = {
     8: "HV_ERR_NO_DEVICE", 9: "HV_ERR_LAUNCH", 10: "HV_ERR_DEVICE_TIMEOUT", 11: "HV_ERR_WORKSPACE",
     12: "HV_ERR_NOALLOC_LIMIT",
 }
-EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", "hv_attn_workspace_bytes",
+EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", "hv_attn_forward_qknorm",
+            "hv_attn_forward_qknorm_ws", "hv_attn_workspace_bytes",
             "hv_video_tokens",
             "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
 
@@ -52,6 +53,14 @@ def lib() -> ctypes.CDLL:
         L.hv_attn_forward_noalloc.restype = ctypes.c_int
         L.hv_attn_forward_noalloc.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
             ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
+        L.hv_attn_forward_qknorm.restype = ctypes.c_int
+        L.hv_attn_forward_qknorm.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_float,
+            ctypes.c_void_p]
+        L.hv_attn_forward_qknorm_ws.restype = ctypes.c_int
+        L.hv_attn_forward_qknorm_ws.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_float,
+            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
@@ -166,6 +175,63 @@ def attn_forward_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, tex
                                       ctypes.c_void_p(stream.cuda_stream))
     if st != HV_OK:
         raise HVError(st, "hv_attn_forward_ws")
+    return out
+
+
+def _check_gamma(g: torch.Tensor, device) -> None:
+    if not isinstance(g, torch.Tensor) or not g.is_cuda or g.device != device:
+        raise TypeError("qk_gamma must be a CUDA tensor on the device of q")
+    if g.dtype != torch.float32 or not g.is_contiguous() or tuple(g.shape) != (4, 128):
+        raise ValueError("qk_gamma must be contiguous float32 [4, 128] (Q video, K video, Q text, K text)")
+
+
+def attn_forward_qknorm(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, text_valid,
+                        qk_gamma: torch.Tensor, qk_eps: float = 1e-6, rope_theta: float = 256.0,
+                        scale: float | None = None, out: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, use_workspace: bool = False,
+                        stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Joint 3D-RoPE attention with the per-head QK RMSNorm prologue.
+
+    ``qk_gamma``: float32 [4, 128] CUDA tensor (Q video, K video, Q text,
+    K text). ``use_workspace`` (or a ``workspace`` tensor) selects the
+    two-stage path; its output is bit-identical.
+    """
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    _check_gamma(qk_gamma, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    b_sz, _, heads, _ = q.shape
+    t_lat, hp, wp = (int(x) for x in grid)
+    if len(text_valid) != b_sz:
+        raise ValueError("text_valid needs one entry per batch sample")
+    valid = (ctypes.c_int * b_sz)(*[int(x) for x in text_valid])
+    if scale is None:
+        scale = 1.0 / math.sqrt(128)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    two_stage = use_workspace or workspace is not None
+    if two_stage and workspace is None:
+        workspace = torch.empty(max(workspace_bytes(b_sz, heads, grid, text_len), 0) // 2, dtype=torch.bfloat16,
+                                device=q.device)
+    with torch.cuda.device(q.device):
+        if two_stage:
+            if not workspace.is_cuda or not workspace.is_contiguous():
+                raise ValueError("workspace must be a contiguous CUDA tensor")
+            st = lib().hv_attn_forward_qknorm_ws(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b_sz, heads, t_lat, hp, wp,
+                int(text_len), valid, float(rope_theta), float(scale), qk_gamma.data_ptr(), float(qk_eps),
+                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                ctypes.c_void_p(stream.cuda_stream))
+        else:
+            st = lib().hv_attn_forward_qknorm(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b_sz, heads, t_lat, hp, wp,
+                int(text_len), valid, float(rope_theta), float(scale), qk_gamma.data_ptr(), float(qk_eps),
+                ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_forward_qknorm_ws" if two_stage else "hv_attn_forward_qknorm")
     return out
 
 

@@ -101,9 +101,32 @@ def test_workspace_entry_points(lib):
     assert f(0x10000, 0x20000, 0x30000, 0x40000, 0, 2, 2, 4, 4, 8, valid, 256.0, 0.088, 0x90000, 1 << 20, None) == 3
 
 
+def test_qknorm_entry_points_validate_arguments(lib):
+    valid = (ctypes.c_int * 1)(5)
+    f, fw = lib.hv_attn_forward_qknorm, lib.hv_attn_forward_qknorm_ws
+    base = (0x10000, 0x20000, 0x30000, 0x40000, 1, 2, 2, 4, 4, 8, valid, 256.0, 0.088)
+    g = 0x900000
+    assert f(*base, None, 1e-6, None) == 1                      # gamma missing
+    assert f(*base, g + 4, 1e-6, None) == 2                     # gamma misaligned
+    assert f(*base, g, -1e-6, None) == 7                        # eps < 0
+    assert f(*base, g, float("nan"), None) == 7
+    assert f(*base, 0x40000 + 64, 1e-6, None) == 6              # gamma inside out
+    assert f(*base, 0x40000 - 1024, 1e-6, None) == 6            # gamma running into out
+    # shape and text errors come first, as in hv_attn_forward
+    assert f(0x10000, 0x20000, 0x30000, 0x40000, 0, 2, 2, 4, 4, 8, valid, 256.0, 0.088, g, 1e-6, None) == 3
+    # the workspace variant checks the same arguments first (its workspace is
+    # looked at after the device check, in the GPU tests)
+    assert fw(*base, None, 1e-6, 0x800000, 1 << 20, None) == 1
+    assert fw(*base, g, float("inf"), 0x800000, 1 << 20, None) == 7
+
+
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     import torch
     if torch.cuda.is_available():
         pytest.skip("a GPU is present; covered by the gpu tests")
     st = _call(lib, q=1 << 32, k=2 << 32, v=3 << 32, out=4 << 32)
+    assert st in (8, 9)
+    valid = (ctypes.c_int * 1)(5)
+    st = lib.hv_attn_forward_qknorm(1 << 32, 2 << 32, 3 << 32, 4 << 32, 1, 2, 2, 4, 4, 8, valid, 256.0, 0.088,
+                                    5 << 32, 1e-6, None)
     assert st in (8, 9)
