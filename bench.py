@@ -62,6 +62,7 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiling runs)")
     ap.add_argument("--no-ws", action="store_true", help="skip timing the workspace (pre-rotated K) path")
+    ap.add_argument("--no-qknorm", action="store_true", help="skip timing the QK RMSNorm prologue paths")
     return ap.parse_args()
 
 
@@ -343,6 +344,33 @@ def run_ours(args, wl, inp, rank, world, local):
                            "kernel, then the attention kernel rotating Q on load; output bit-identical"}
         del ws
 
+    # the QK RMSNorm prologue (seeded gammas), one-kernel and two-stage forms
+    qk_line = None
+    if not args.no_qknorm:
+        gam = torch.from_numpy(np.random.default_rng(1234).uniform(0.5, 1.5, (4, 128)).astype(np.float32)).to(dev)
+        ws = torch.empty(H.workspace_bytes(wl.batch, wl.heads, wl.grid, wl.text_len) // 2, dtype=torch.bfloat16,
+                         device=dev)
+        qk_line = {"unit": UNIT, "what": "hv_attn_forward_qknorm / _qknorm_ws: per-head RMSNorm of Q and K "
+                                         "(video and text gammas, eps 1e-6) before the rotation"}
+        for key, wsp in (("fused", None), ("workspace", ws)):
+            call = lambda: H.attn_forward_qknorm(q, k, v, wl.grid, wl.text_len, text_valid, gam, 1e-6, out=out,
+                                                 workspace=wsp, stream=stream)
+            for _ in range(max(1, args.warmup)):
+                call()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(args.steps):
+                call()
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            if H.last_device_error() != 0:
+                raise RuntimeError("device error in the QK-norm path")
+            q_ms, q_value = replica_throughput(a0.elapsed_time(a1) / args.steps, flops, world)
+            qk_line[key] = {"value": q_value, "ms_per_step": q_ms}
+        del ws
+
     # end to end through the host-buffer API: pinned host in, pinned host out
     e2e = None
     if not args.no_e2e:
@@ -387,6 +415,7 @@ def run_ours(args, wl, inp, rank, world, local):
         "gpu_launches": args.steps,
         "clocks": clk,
         "workspace_path": ws_line,
+        "qk_norm_path": qk_line,
     }
     if world == 1 and not args.no_cpu_baseline:
         cpu_value, info = oracle_sample(wl, inp, args.cpu_seconds)
