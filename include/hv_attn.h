@@ -190,6 +190,48 @@ int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* o
                             float rope_theta, float scale, void* cuda_stream);
 
 /*
+ * hv_attn_forward_host - the whole call from and to HOST memory, with the
+ * copies overlapping the attention kernel. The heads are cut into
+ * `head_groups` groups (heads % head_groups == 0); per group, in a pipeline
+ * of two device staging slots: a 2-D copy of the group's q, k, v columns
+ * host -> device, hv_attn_forward on the contiguous [B, S, heads/groups, 128]
+ * staging tensors, and a 2-D copy of the group's output columns back into
+ * out_host. Heads are independent (§5.2 computes attention per head), so the
+ * result equals hv_attn_forward's bit for bit. No counterpart in the pages:
+ * it is the host-buffer form of the same call.
+ *
+ * q_host, k_host, v_host, out_host: HOST pointers, layout as hv_attn_forward;
+ *            page-locked (pinned) memory lets the copies run asynchronously;
+ *            out_host must not overlap the inputs.
+ * head_groups: >= 1, dividing heads (1 = no overlap, copies and compute in turn).
+ * workspace: DEVICE pointer, 16-byte aligned, at least
+ *            hv_attn_host_workspace_bytes(...) bytes, owned by the caller.
+ * cuda_stream: the kernels run on it; the copies run on two streams the
+ *            library creates once per device (make the first call before any
+ *            stream capture). The call is asynchronous: `cuda_stream` is made to
+ *            wait for the last copy, so out_host is complete once that stream
+ *            has been synchronised; the host buffers must stay valid until then.
+ *            Calls on one device share the copy streams and are enqueued one
+ *            at a time (a mutex), so they run in turn.
+ * Errors: HV_ERR_NULL_POINTER, HV_ERR_BAD_SHAPE (also bad head_groups),
+ * HV_ERR_BAD_TEXT, HV_ERR_ALIAS (host buffers), HV_ERR_WORKSPACE, and those of
+ * hv_attn_forward for one group's call; HV_ERR_LAUNCH if a copy or a stream
+ * operation fails.
+ */
+int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                         int B, int heads, int T, int Hp, int Wp,
+                         int text_len, const int* text_valid,
+                         float rope_theta, float scale, int head_groups,
+                         void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * hv_attn_host_workspace_bytes - device workspace hv_attn_forward_host needs:
+ * 8 * B * S * (heads / head_groups) * 128 * 2 bytes (two slots of q, k, v, out);
+ * -1 for a bad shape or head_groups.
+ */
+long long hv_attn_host_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len, int head_groups);
+
+/*
  * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)
  * of an F x H x W clip (§4 "Causal 3D VAE": temporal compression 4 keeping the
  * first frame, spatial 8, then the 1x2x2 patch). Returns -1 when F is not

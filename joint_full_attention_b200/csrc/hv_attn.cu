@@ -768,14 +768,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     for (int e = 0; e < BN; ++e)
                         if (e >= c.last_lim) sr[e] = __float_as_uint(-INFINITY);
                 }
-                float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-                float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+                // row max, two columns per (three-input) max instruction
+                float mx0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[4]));
+                float mx1 = fmaxf(__uint_as_float(sr[1]), __uint_as_float(sr[5]));
+                float mx2 = fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[6]));
+                float mx3 = fmaxf(__uint_as_float(sr[3]), __uint_as_float(sr[7]));
 #pragma unroll
-                for (int e = 4; e < BN; e += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(sr[e]));
-                    mx1 = fmaxf(mx1, __uint_as_float(sr[e + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(sr[e + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(sr[e + 3]));
+                for (int e = 8; e < BN; e += 8) {
+                    mx0 = fmax3(mx0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 4]));
+                    mx1 = fmax3(mx1, __uint_as_float(sr[e + 1]), __uint_as_float(sr[e + 5]));
+                    mx2 = fmax3(mx2, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 6]));
+                    mx3 = fmax3(mx3, __uint_as_float(sr[e + 3]), __uint_as_float(sr[e + 7]));
                 }
                 const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
                 float m_new = m, alpha = 1.f;
@@ -1146,6 +1149,42 @@ static int launch_rope_k(const Call& call, const void* k, void* dst, int heads, 
     return cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
+// Streams and events of the host-buffer pipeline, created once per device.
+struct HostPipe {
+    bool ok = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+};
+
+static std::mutex g_host_pipe_mu;   // also serialises the enqueue of whole calls
+
+static HostPipe* host_pipe(int dev) {
+    static HostPipe pipes[64];
+    HostPipe& hp = pipes[dev & 63];
+    if (!hp.ok) {
+        bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; i < 2 && good; ++i)
+            good = cudaEventCreateWithFlags(&hp.h2d_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&hp.d2h_done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) return nullptr;
+        hp.ok = true;
+    }
+    return &hp;
+}
+
+// bytes of one head group's staging tensor [B, S, heads/groups, 128] bf16
+static long long host_group_bytes(int B, int heads, int T, int Hp, int Wp, int text_len, int groups) {
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || text_len < 0 || text_len > HV_MAX_TEXT_LEN ||
+        groups < 1 || heads % groups != 0)
+        return -1;
+    const long long s_len = static_cast<long long>(T) * Hp * Wp + text_len;
+    return static_cast<long long>(B) * s_len * (heads / groups) * D * 2;
+}
+
 }  // namespace hv
 
 extern "C" {
@@ -1262,6 +1301,75 @@ int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* o
     if (st != HV_OK) return st;
     return launch_attention(call, q, scratch, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale,
                             true, nullptr, 0.f, stream);
+}
+
+long long hv_attn_host_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len, int head_groups) {
+    const long long g = hv::host_group_bytes(B, heads, T, Hp, Wp, text_len, head_groups);
+    return g < 0 ? -1 : 8 * g;   // two slots of q, k, v, out
+}
+
+int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_host, void* out_host, int B,
+                         int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
+                         float scale, int head_groups, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    using namespace hv;
+    if (!q_host || !k_host || !v_host || !out_host || !text_valid || !workspace) return HV_ERR_NULL_POINTER;
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH || head_groups < 1 ||
+        heads % head_groups != 0)
+        return HV_ERR_BAD_SHAPE;
+    const long long gbytes = host_group_bytes(B, heads, T, Hp, Wp, text_len, head_groups);
+    if (gbytes < 0) return HV_ERR_BAD_TEXT;
+    const int hg = heads / head_groups;
+    const size_t full = static_cast<size_t>(gbytes) * head_groups;
+    if (overlaps(out_host, q_host, full) || overlaps(out_host, k_host, full) || overlaps(out_host, v_host, full))
+        return HV_ERR_ALIAS;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) || workspace_bytes < static_cast<size_t>(8 * gbytes))
+        return HV_ERR_WORKSPACE;
+    // validate one group's device call up front (shapes, text, scalars, device)
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto slot_buf = [&](int slot, int t) { return ws + (static_cast<size_t>(slot) * 4 + t) * gbytes; };
+    Call call;
+    int st = validate(slot_buf(0, 0), slot_buf(0, 1), slot_buf(0, 2), slot_buf(0, 3), B, hg, T, Hp, Wp, text_len,
+                      text_valid, rope_theta, scale, call);
+    if (st != HV_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_host_pipe_mu);
+    HostPipe* hp = host_pipe(dev);
+    if (!hp) return HV_ERR_LAUNCH;
+    const cudaStream_t cs = static_cast<cudaStream_t>(cuda_stream);
+    const size_t row = static_cast<size_t>(heads) * D * 2, grow = static_cast<size_t>(hg) * D * 2;
+    const size_t rows = static_cast<size_t>(B) * call.S;
+    bool good = cudaEventRecord(hp->start, cs) == cudaSuccess &&
+                cudaStreamWaitEvent(hp->h2d, hp->start, 0) == cudaSuccess &&
+                cudaStreamWaitEvent(hp->d2h, hp->start, 0) == cudaSuccess;
+    const void* src[3] = {q_host, k_host, v_host};
+    for (int g = 0; g < head_groups && good; ++g) {
+        const int slot = g & 1;
+        const size_t col = static_cast<size_t>(g) * grow;
+        // inputs of this group into the slot, once the group that used it last has been computed
+        good = cudaStreamWaitEvent(hp->h2d, hp->comp_done[slot], 0) == cudaSuccess;
+        for (int t = 0; t < 3 && good; ++t)
+            good = cudaMemcpy2DAsync(slot_buf(slot, t), grow, static_cast<const uint8_t*>(src[t]) + col, row, grow,
+                                     rows, cudaMemcpyHostToDevice, hp->h2d) == cudaSuccess;
+        good = good && cudaEventRecord(hp->h2d_done[slot], hp->h2d) == cudaSuccess;
+        // attention of the group, once its inputs are in and the slot's output has been copied out
+        good = good && cudaStreamWaitEvent(cs, hp->h2d_done[slot], 0) == cudaSuccess &&
+               cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
+        if (good) {
+            st = launch_attention(call, slot_buf(slot, 0), slot_buf(slot, 1), slot_buf(slot, 2), slot_buf(slot, 3), B,
+                                  hg, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false, nullptr, 0.f, cs);
+            if (st != HV_OK) return st;
+        }
+        good = good && cudaEventRecord(hp->comp_done[slot], cs) == cudaSuccess;
+        // the group's output back into its columns of out_host
+        good = good && cudaStreamWaitEvent(hp->d2h, hp->comp_done[slot], 0) == cudaSuccess &&
+               cudaMemcpy2DAsync(static_cast<uint8_t*>(out_host) + col, row, slot_buf(slot, 3), grow, grow, rows,
+                                 cudaMemcpyDeviceToHost, hp->d2h) == cudaSuccess &&
+               cudaEventRecord(hp->d2h_done[slot], hp->d2h) == cudaSuccess;
+    }
+    // the caller's stream completes after the last copy out
+    for (int slot = 0; slot < 2 && good; ++slot) good = cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
+    return good ? HV_OK : HV_ERR_LAUNCH;
 }
 
 int hv_attn_last_device_error(void) {

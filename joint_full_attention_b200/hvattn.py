@@ -18,6 +18,7 @@ _LIB_PATH = Path(__file__).resolve().parent / "libhvattn.so"
 _lib = None
 
 HV_OK = 0
+HV_ERR_BAD_SHAPE = 3
 STATUS_NAMES = {
     0: "HV_OK", 1: "HV_ERR_NULL_POINTER", 2: "HV_ERR_MISALIGNED", 3: "HV_ERR_BAD_SHAPE",
     4: "HV_ERR_BAD_TEXT", 5: "HV_ERR_TOO_LARGE", 6: "HV_ERR_ALIAS", 7: "HV_ERR_BAD_SCALAR",
@@ -25,7 +26,8 @@ STATUS_NAMES = {
     12: "HV_ERR_NOALLOC_LIMIT",
 }
 EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", "hv_attn_forward_qknorm",
-            "hv_attn_forward_qknorm_ws", "hv_attn_workspace_bytes",
+            "hv_attn_forward_qknorm_ws", "hv_attn_forward_host", "hv_attn_host_workspace_bytes",
+            "hv_attn_workspace_bytes",
             "hv_video_tokens",
             "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
 
@@ -61,6 +63,12 @@ def lib() -> ctypes.CDLL:
         L.hv_attn_forward_qknorm_ws.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
             ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_float,
             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        L.hv_attn_forward_host.restype = ctypes.c_int
+        L.hv_attn_forward_host.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_size_t, ctypes.c_void_p]
+        L.hv_attn_host_workspace_bytes.restype = ctypes.c_longlong
+        L.hv_attn_host_workspace_bytes.argtypes = [ctypes.c_int] * 7
         L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
@@ -235,28 +243,57 @@ def attn_forward_qknorm(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid,
     return out
 
 
+def default_head_groups(heads: int) -> int:
+    """Head groups of the host-buffer pipeline: the largest of 8, 6, 4, 3, 2
+    that divides the heads (at 720p 8 groups left 5 ms of copies exposed, 1
+    group 48 ms)."""
+    for g in (8, 6, 4, 3, 2):
+        if heads % g == 0:
+            return g
+    return 1
+
+
 def attn_forward_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, grid, text_len: int,
                       text_valid, rope_theta: float = 256.0, scale: float | None = None,
                       device: int | torch.device = 0, out_host: torch.Tensor | None = None,
-                      work: dict | None = None) -> torch.Tensor:
-    """Host-to-host call: copy pinned host inputs to the GPU, run, copy the output back.
+                      work: dict | None = None, head_groups: int | None = None) -> torch.Tensor:
+    """Host-to-host call (``hv_attn_forward_host``): pinned host inputs in, output back in host memory.
 
-    ``work`` may hold reusable device buffers (keys "q", "k", "v", "out") so
-    that repeated calls allocate nothing on the device.
+    The library pipelines per head group: copy in, attention, copy out, with
+    the copies overlapping the kernels. ``work`` may hold the reusable device
+    workspace (key "host_ws") so that repeated calls allocate nothing on the
+    device. Returns after the output is in ``out_host``.
     """
     dev = torch.device("cuda", device) if isinstance(device, int) else device
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4 or t.shape[-1] != 128:
+            raise ValueError(f"{name} must be a contiguous bfloat16 host tensor [B, S, heads, 128]")
+        if tuple(t.shape) != tuple(q_host.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} != {tuple(q_host.shape)}")
+    b_sz, _, heads, _ = q_host.shape
+    if len(text_valid) != b_sz:
+        raise ValueError("text_valid needs one entry per batch sample")
+    groups = default_head_groups(heads) if head_groups is None else int(head_groups)
+    t_lat, hp, wp = (int(x) for x in grid)
+    need = int(lib().hv_attn_host_workspace_bytes(b_sz, heads, t_lat, hp, wp, int(text_len), groups))
+    if need < 0:
+        raise HVError(HV_ERR_BAD_SHAPE, "hv_attn_host_workspace_bytes")
     work = {} if work is None else work
-    for name, src in (("q", q_host), ("k", k_host), ("v", v_host)):
-        buf = work.get(name)
-        if buf is None or buf.shape != src.shape:
-            buf = work[name] = torch.empty(src.shape, dtype=src.dtype, device=dev)
-        buf.copy_(src, non_blocking=True)
-    o = work.get("out")
-    if o is None or o.shape != q_host.shape:
-        o = work["out"] = torch.empty(q_host.shape, dtype=q_host.dtype, device=dev)
-    attn_forward(work["q"], work["k"], work["v"], grid, text_len, text_valid, rope_theta, scale, out=o)
+    ws = work.get("host_ws")
+    if ws is None or ws.device != dev or ws.numel() * ws.element_size() < need:
+        ws = work["host_ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
     if out_host is None:
         out_host = torch.empty(q_host.shape, dtype=q_host.dtype, pin_memory=True)
-    out_host.copy_(o, non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
+    valid = (ctypes.c_int * b_sz)(*[int(x) for x in text_valid])
+    if scale is None:
+        scale = 1.0 / math.sqrt(128)
+    stream = torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        st = lib().hv_attn_forward_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                        out_host.data_ptr(), b_sz, heads, t_lat, hp, wp, int(text_len), valid,
+                                        float(rope_theta), float(scale), groups, ws.data_ptr(),
+                                        ws.numel() * ws.element_size(), ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_forward_host")
+    stream.synchronize()
     return out_host

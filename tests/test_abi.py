@@ -120,6 +120,22 @@ def test_qknorm_entry_points_validate_arguments(lib):
     assert fw(*base, g, float("inf"), 0x800000, 1 << 20, None) == 7
 
 
+def test_host_entry_point_validates_arguments(lib):
+    assert lib.hv_attn_host_workspace_bytes(1, 24, 33, 45, 80, 256, 4) == 8 * 119056 * 6 * 256
+    assert lib.hv_attn_host_workspace_bytes(1, 24, 33, 45, 80, 256, 5) == -1     # 5 does not divide 24
+    assert lib.hv_attn_host_workspace_bytes(1, 24, 33, 45, 80, 256, 0) == -1
+    valid = (ctypes.c_int * 1)(5)
+    f = lib.hv_attn_forward_host
+    hq, hk, hv, ho = 1 << 30, 2 << 30, 3 << 30, 4 << 30
+    args = (1, 2, 2, 4, 4, 8, valid, 256.0, 0.088)
+    assert f(None, hk, hv, ho, *args, 2, 0x900000, 1 << 20, None) == 1
+    assert f(hq, hk, hv, ho, *args, 2, None, 1 << 20, None) == 1
+    assert f(hq, hk, hv, ho, *args, 3, 0x900000, 1 << 20, None) == 3          # 3 does not divide 2 heads
+    assert f(hq, hk, hv, hq + 64, *args, 1, 0x900000, 1 << 20, None) == 6     # out over q
+    assert f(hq, hk, hv, ho, *args, 2, 0x900008, 1 << 20, None) == 11         # misaligned workspace
+    assert f(hq, hk, hv, ho, *args, 2, 0x900000, 1000, None) == 11            # too small
+
+
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     import torch
     if torch.cuda.is_available():

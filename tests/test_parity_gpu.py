@@ -238,3 +238,25 @@ def test_workspace_errors():
         H.attn_forward_ws(q, q, q, (2, 4, 4), 8, [5], out=torch.empty_like(q), workspace=q.view(-1))
     assert e.value.status == 11
     assert H.last_device_error() == 0
+
+
+# ------------------------------------------------------- host-buffer pipeline
+
+@pytest.mark.parametrize("name,groups,pinned", [("img256", 1, True), ("img256", 4, True), ("img256", 24, False),
+                                                ("v544x960x17", 3, True), ("v544x960x17", 8, False)])
+def test_host_pipeline_bit_identical(name, groups, pinned):
+    """hv_attn_forward_host (per-head-group copies overlapping the kernels)
+    returns exactly what hv_attn_forward computes on device buffers."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, seed=6)
+    q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
+    ref = H.attn_forward(q, k, v, wl.grid, wl.text_len, inp["text_valid"]).cpu()
+    host = []
+    for n in ("q", "k", "v"):
+        t = torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16)
+        host.append(t.pin_memory() if pinned else t.clone())
+    work = {}
+    for _ in range(2):      # the second call reuses the workspace and the copy streams
+        out = H.attn_forward_host(*host, wl.grid, wl.text_len, inp["text_valid"], work=work, head_groups=groups)
+        assert torch.equal(out, ref)
+    assert H.last_device_error() == 0
