@@ -57,6 +57,10 @@ Readings where the pages are silent (each also listed in the design doc):
   R14 video rows take the video stream's gamma, text rows the text stream's
      ([P1] §5.2: the double-stream blocks keep separate parameters per
      modality); a single-stream block passes the same gamma twice.
+  R16 ring-attention blocks ([P1] §9.2): a query or key block is a run of
+     consecutive joint-sequence rows given by its count of leading video rows
+     and the global token index of the first; results of disjoint key blocks
+     combine through their per-row log-sum-exp (the softmax over the union).
   R15 order: RMSNorm first, then the 3D rotation of the video rows (the norm
      acts on Q, K as projected, §5.4; RoPE rotates the Q, K that attention
      uses, §5.5). eps is a parameter (the pages give none).
@@ -281,6 +285,67 @@ def joint_attention_samples(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: t
         out[sel] = joint_attention_head(q[b, :, h], k[b, :, h], v[b, :, h], grid,
                                         int(text_valid[b]), theta, scale, rows=samples[sel, 2], qk_norm=qk_norm)
     return out
+
+
+def joint_attention_block(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: tuple[int, int, int],
+                          q_video: int, q_pos0: int, k_video: int, k_pos0: int, kv_len: int,
+                          theta: float = DEFAULT_THETA, scale: float | None = None,
+                          qk_norm: dict | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """Attention of a block of query rows against a block of key rows, with
+    the log-sum-exp of each row: the step of ring attention ([P1] §9.2: each
+    rank keeps a segment of queries while K/V blocks pass around the ring).
+
+    Reading R16: a block holds a run of consecutive joint-sequence rows; its
+    first ``*_video`` rows are video tokens whose global token indices start at
+    ``*_pos0`` (rotated by the 3D RoPE of those tokens, R4/R6), the rest are
+    text rows (not rotated). Only the first ``kv_len`` key rows take part.
+    Returns O = softmax(scores) V over those keys and
+    lse = log(sum_j exp(score_j)) (natural log of the scaled scores), per row;
+    a block with kv_len = 0 gives O = 0 and lse = -inf (it contributes
+    nothing when merged).
+
+    q: (Sq, 128), k, v: (Sk, 128) for one (batch, head).
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    t_lat, hp, wp = grid
+    pos = token_positions(t_lat, hp, wp)
+    qr = np.asarray(q, dtype=np.float64).copy()
+    kr = np.asarray(k, dtype=np.float64)[:kv_len].copy()
+    vv = np.asarray(v, dtype=np.float64)[:kv_len]
+    if qk_norm is not None:
+        eps = float(qk_norm["eps"])
+        qr = qk_norm_rows(qr, np.arange(qr.shape[0]) < q_video, qk_norm["gamma_q_video"],
+                          qk_norm["gamma_q_text"], eps)
+        kr = qk_norm_rows(kr, np.arange(kv_len) < k_video, qk_norm["gamma_k_video"], qk_norm["gamma_k_text"], eps)
+    if q_video > 0:
+        qr[:q_video] = rope3d_rotate(qr[:q_video], pos[q_pos0:q_pos0 + q_video], theta)
+    kv_vid = min(k_video, kv_len)
+    if kv_vid > 0:
+        kr[:kv_vid] = rope3d_rotate(kr[:kv_vid], pos[k_pos0:k_pos0 + kv_vid], theta)
+    if kv_len == 0:
+        return np.zeros_like(qr), np.full(qr.shape[0], -np.inf)
+    scores = (qr @ kr.T) * scale
+    mx = scores.max(axis=1, keepdims=True)
+    p = np.exp(scores - mx)
+    tot = p.sum(axis=1, keepdims=True)
+    return (p / tot) @ vv, (mx + np.log(tot))[:, 0]
+
+
+def merge_blocks(outs, lses) -> tuple[np.ndarray, np.ndarray]:
+    """Combine the results of disjoint key blocks of the same query rows:
+    O = sum_i exp(lse_i - lse) O_i with lse = log(sum_i exp(lse_i))
+    (the softmax over the union of the blocks' keys)."""
+    lses = np.stack([np.asarray(x, dtype=np.float64) for x in lses])       # (blocks, rows)
+    top = lses.max(axis=0)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w = np.exp(lses - safe)                                                # (blocks, rows)
+    tot = w.sum(axis=0)
+    out = sum(w[i][:, None] * np.asarray(o, dtype=np.float64) for i, o in enumerate(outs))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(tot[:, None] > 0, out / np.where(tot > 0, tot, 1.0)[:, None], 0.0)
+        lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return out, lse
 
 
 def attention_flops(batch: int, heads: int, grid: tuple[int, int, int], text_len: int, text_valid) -> float:
