@@ -232,6 +232,51 @@ int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_h
 long long hv_attn_host_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len, int head_groups);
 
 /*
+ * hv_attn_forward_block - one step of ring attention (§9.2 "xDiT/USP 序列并行":
+ * each rank keeps a run of query rows while K/V blocks pass around the ring):
+ * attention of a block of Sq query rows against a block of Sk key/value rows,
+ * plus the log-sum-exp of every query row, so that the results of several
+ * key blocks can be merged (hv_attn_merge).
+ *
+ * Both blocks are runs of consecutive rows of the joint sequence of the
+ * T x Hp x Wp grid: the first q_video (k_video) rows are video tokens whose
+ * global token indices are q_pos0, q_pos0 + 1, ... (k_pos0, ...), rotated by
+ * the 3D RoPE of those tokens; the remaining rows are text (not rotated).
+ * Only the first kv_len[b] key rows of sample b take part.
+ *
+ * q, out   : device bf16 [B, Sq, heads, 128]; k, v: device bf16 [B, Sk, heads, 128].
+ * lse      : device fp32 [B, Sq, heads] or NULL; lse = log(sum_j exp(s_j)) of
+ *            the scaled scores s_j = scale * q'.k'_j over the block's keys.
+ * kv_len   : HOST pointer to B ints, 1 <= kv_len[b] <= Sk (a block with no
+ *            key at all has no result; leave it out of the merge).
+ * Constraints: 0 <= q_video <= Sq, 0 <= k_video <= Sk, q_pos0, k_pos0 >= 0 and
+ * q_pos0 + q_video, k_pos0 + k_video <= T*Hp*Wp (HV_ERR_BAD_SHAPE otherwise);
+ * kv_len out of range: HV_ERR_BAD_TEXT; out or lse overlapping an input or
+ * each other: HV_ERR_ALIAS. Other errors, ownership and asynchrony as
+ * hv_attn_forward. hv_attn_forward is the special case Sq = Sk = S,
+ * q_video = k_video = N, offsets 0, kv_len[b] = N + text_valid[b].
+ */
+int hv_attn_forward_block(const void* q, const void* k, const void* v, void* out, float* lse,
+                          int B, int heads, int T, int Hp, int Wp,
+                          int Sq, int q_video, int q_pos0, int Sk, int k_video, int k_pos0,
+                          const int* kv_len, float rope_theta, float scale, void* cuda_stream);
+
+/*
+ * hv_attn_merge - fold one key block's result (o_part bf16, lse_part fp32)
+ * into the running result (o_acc fp32, lse_acc fp32) of the same `rows` query
+ * rows of 128 channels: with m = max(lse_acc, lse_part), w = exp(lse - m),
+ *   o_acc <- (w_acc o_acc + w_part o_part) / (w_acc + w_part),
+ *   lse_acc <- m + log(w_acc + w_part),
+ * the softmax over the union of the keys. Start from o_acc = 0 and
+ * lse_acc = -inf. If `out` is not NULL the merged rows are also written to it
+ * as bf16 (the last merge of a ring). Device pointers; o_acc 16-byte, o_part and
+ * out 8-byte, lse 4-byte aligned. Asynchronous on cuda_stream. No
+ * counterpart in the pages beyond the merge rule of ring attention.
+ */
+int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* out,
+                  long long rows, void* cuda_stream);
+
+/*
  * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)
  * of an F x H x W clip (§4 "Causal 3D VAE": temporal compression 4 keeping the
  * first frame, spatial 8, then the 1x2x2 patch). Returns -1 when F is not

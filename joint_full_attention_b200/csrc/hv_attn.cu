@@ -142,7 +142,15 @@ struct __align__(64) Params {
     float theta_log2;   // log2(rope_theta)
     float scale_log2;   // scale * log2(e)
     unsigned long long timeout_ns;
-    int text_valid[HV_MAX_BATCH];
+    // Geometry of the row blocks. The standard call: Q and K/V are the whole
+    // joint sequence (Sk = S, q_vid = k_vid = N, offsets 0). A ring-attention
+    // block: Q rows and K/V rows are runs of the joint sequence whose first
+    // q_vid / k_vid rows are video tokens with global token indices starting
+    // at q_pos0 / k_pos0; the other rows are text.
+    int Sk;             // rows of the K and V tensors (S: rows of Q and out)
+    int q_vid, q_pos0, k_vid, k_pos0;
+    float* lse;         // optional [B, S, H] fp32: natural-log log-sum-exp of each row's scaled scores
+    int kv_len[HV_MAX_BATCH];   // keys taking part, per batch sample (the rest are masked)
 };
 
 __device__ unsigned int g_dev_error = 0;
@@ -200,7 +208,7 @@ __device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
     const int bh = u / p.n_qunits;
     c.h = bh % p.H;
     c.b = bh / p.H;
-    const int kv_len = p.N + p.text_valid[c.b];
+    const int kv_len = p.kv_len[c.b];
     c.nt = (kv_len + BN - 1) / BN;
     c.last_lim = kv_len - (c.nt - 1) * BN;
     return c;
@@ -338,14 +346,17 @@ __device__ __forceinline__ void advance8(GridPos& g, const Params& p) {
     }
 }
 
-__device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int rt, const RopeLane& L,
-                                          const Params& p) {
+// Rows n0 + rb, n0 + rb + 12, ... of a tile; local rows below `vid` are video
+// tokens whose global token index is pos0 + row (the rest are text, left as
+// they are).
+__device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int vid, int pos0, int rt,
+                                          const RopeLane& L, const Params& p) {
     const int rb = rt >> 4;
     int n = n0 + rb;
-    if (n >= p.N) return;
+    if (n >= vid) return;
     GridPos g;
-    g.w = n % p.Wp;
-    const int th = n / p.Wp;
+    g.w = (pos0 + n) % p.Wp;
+    const int th = (pos0 + n) / p.Wp;
     g.h = th % p.Hp;
     g.t = th / p.Hp;
     const uint32_t box_base = tile + L.box * BOX_BYTES;
@@ -358,7 +369,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 #pragma unroll 1
         for (int r = rb; r < BM; r += 2 * ROPE_GROUPS) {
             const int pos0 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
-            const bool has1 = n + ROPE_GROUPS < p.N && r + ROPE_GROUPS < BM;
+            const bool has1 = n + ROPE_GROUPS < vid && r + ROPE_GROUPS < BM;
             advance8(g, p);
             const int pos1 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
             const uint32_t a0 = row_addr(r);
@@ -378,7 +389,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
             if (!has1) break;
             sts128(a1, rotate_chunk(d1, c1, s1));
             n += 2 * ROPE_GROUPS;
-            if (n >= p.N) break;   // rows only grow: the rest are text or past the end
+            if (n >= vid) break;   // rows only grow: the rest are text or past the end
             advance8(g, p);
         }
     } else {
@@ -396,7 +407,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
             }
             sts128(a, make_uint4(wv[0], wv[1], wv[2], wv[3]));
             n += ROPE_GROUPS;
-            if (n >= p.N) break;
+            if (n >= vid) break;
             advance8(g, p);
         }
     }
@@ -410,12 +421,13 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 // iterations (rb and rb + 1 share a warp and a trip count), as the row sum is
 // a half-warp shuffle.
 __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
-                                               int n0, int rt, const RopeLane& L, const Params& p) {
+                                               int n0, int vid, int pos0, int rt, const RopeLane& L,
+                                               const Params& p) {
     const int rb = rt >> 4;
     int n = n0 + rb;
     GridPos g;
-    g.w = n % p.Wp;
-    const int th = n / p.Wp;
+    g.w = (pos0 + n) % p.Wp;
+    const int th = (pos0 + n) / p.Wp;
     g.h = th % p.Hp;
     g.t = th / p.Hp;
     const uint32_t box_base = tile + L.box * BOX_BYTES;
@@ -425,7 +437,7 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
     const uint32_t gofs = 4u * static_cast<uint32_t>(L.ch0);
 #pragma unroll 1
     for (int r = rb; r < BM; r += ROPE_GROUPS) {
-        const bool video = n < p.N;
+        const bool video = n < vid;
         const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
         const uint32_t a = box_base + r * 128 + ((L.cin ^ (r & 7)) << 4);
         const uint4 d = lds128(a);
@@ -472,8 +484,11 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
 
 // The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
 // each to the MMA warp.
+template <bool BLOCK>
 __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
                                           uint32_t sK, uint32_t sTable, uint32_t sGamma) {
+    const int q_vid = BLOCK ? p.q_vid : p.N, q_pos0 = BLOCK ? p.q_pos0 : 0;
+    const int k_vid = BLOCK ? p.k_vid : p.N, k_pos0 = BLOCK ? p.k_pos0 : 0;
     const RopeLane L = make_rope_lane(rt, p);
     const int lane = threadIdx.x & 31;
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -485,9 +500,9 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
             if (p.qk_norm)
-                rope_norm_tile(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, rt, L, p);
+                rope_norm_tile(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, q_vid, q_pos0, rt, L, p);
             else
-                rope_tile(sQ + qi * TILE_BYTES, sTable, n0, rt, L, p);
+                rope_tile(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -497,9 +512,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int j = 0; j < c.nt; ++j, kr.next()) {
             if (!(ok = waiter.wait_warp(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
             if (p.qk_norm)
-                rope_norm_tile(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, j * BN, rt, L, p);
-            else if (j * BN < p.N)
-                rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, rt, L, p);
+                rope_norm_tile(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, j * BN, k_vid, k_pos0,
+                               rt, L, p);
+            else if (j * BN < k_vid)
+                rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, k_vid, k_pos0, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
@@ -530,6 +546,10 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
+// BLOCK: a ring-attention block (Q and K/V rows at their own global offsets,
+// log-sum-exp output); the standard call is compiled without that
+// generality (video rows = the first N rows of both, no offsets).
+template <bool BLOCK>
 __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -668,7 +688,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
       } else if (warp > WARP_MMA) {
         // RoPE helpers: threads 128..191 of the RoPE role
-        rope_role(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
+        rope_role<BLOCK>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
@@ -737,7 +757,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     } else if (warp >= WARP_ROPE) {
         regs_decrease<REGS_ROPE>();
         // ------------------------------------------------------------ RoPE
-        rope_role(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
+        rope_role<BLOCK>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -835,6 +855,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             const float inv_l = 1.f / l;
             const int srow = c.qu * UNIT_ROWS + qi * BM + row;
             const bool store = srow < p.S;
+            if constexpr (BLOCK) {
+                if (p.lse != nullptr && store)
+                    p.lse[(static_cast<size_t>(c.b) * p.S + srow) * p.H + c.h] = (m + log2f(l)) * 0.6931471805599453f;
+            }
             uint4* dst = reinterpret_cast<uint4*>(
                 p.out + ((static_cast<size_t>(c.b) * p.S + (store ? srow : 0)) * p.H + c.h) * D);
 #pragma unroll
@@ -873,8 +897,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
 // B*S*heads*256 bytes once. Warps step through whole pairs of rows (16
 // chunks each), so a row's chunks always share a half-warp.
 __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict__ kin, uint4* __restrict__ kout,
-                                                        long long n_chunks, int H, int S, int N, int Hp, int Wp,
-                                                        float theta_log2, const float* __restrict__ gamma_kv,
+                                                        long long n_chunks, int H, int S, int N, int pos0, int Hp,
+                                                        int Wp, float theta_log2, const float* __restrict__ gamma_kv,
                                                         const float* __restrict__ gamma_kt, float eps) {
     const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
     const int lane = threadIdx.x & 31;
@@ -887,15 +911,16 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
         const int cc = lane & 15;
         const long long row = e >> 4;               // (b * S + s) * H + h
         const int s_idx = static_cast<int>((row / H) % S);
-        const bool video = s_idx < N;
+        const bool video = s_idx < N;           // N: leading video rows of this block
+        const int g_idx = pos0 + s_idx;         // global token index of a video row
         const int ch0 = cc * 8;
         int i0, dax, pos;
         if (ch0 < 16) {
-            i0 = ch0 / 2; dax = 16; pos = s_idx / (Hp * Wp);
+            i0 = ch0 / 2; dax = 16; pos = g_idx / (Hp * Wp);
         } else if (ch0 < 72) {
-            i0 = (ch0 - 16) / 2; dax = 56; pos = (s_idx / Wp) % Hp;
+            i0 = (ch0 - 16) / 2; dax = 56; pos = (g_idx / Wp) % Hp;
         } else {
-            i0 = (ch0 - 72) / 2; dax = 56; pos = s_idx % Wp;
+            i0 = (ch0 - 72) / 2; dax = 56; pos = g_idx % Wp;
         }
         if (norm) {
             const float* gsrc = (video ? gamma_kv : gamma_kt) + ch0;
@@ -925,6 +950,44 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
             d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
         if (live) kout[e] = d;
+    }
+}
+
+// Ring attention, merge step: fold the result (o_part, lse_part) of one more
+// key block into the running (o_acc, lse_acc) of the same query rows, as the
+// softmax over the union of the keys: with m = max(lse_acc, lse_part),
+// w = exp(lse - m), o_acc = (w_acc o_acc + w_part o_part) / (w_acc + w_part)
+// and lse_acc = m + log(w_acc + w_part). A block with lse = -inf adds nothing.
+// One warp per 128-channel row; optionally writes the merged row as bf16.
+__global__ void __launch_bounds__(256) hv_merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
+                                                       const uint2* __restrict__ o_part,
+                                                       const float* __restrict__ lse_part, uint2* __restrict__ out,
+                                                       long long rows) {
+    const int lane = threadIdx.x & 31;
+    const long long wpb = blockDim.x >> 5;
+    const long long step = static_cast<long long>(gridDim.x) * wpb;
+    for (long long r = static_cast<long long>(blockIdx.x) * wpb + (threadIdx.x >> 5); r < rows; r += step) {
+        const float la = lse_acc[r], lb = lse_part[r];
+        __syncwarp();
+        const float m = fmaxf(la, lb);
+        float4 a = reinterpret_cast<float4*>(o_acc)[r * 32 + lane];
+        float lse = m;
+        if (m != -INFINITY) {
+            const float wa = expf(la - m), wb = expf(lb - m);
+            const float tot = wa + wb;
+            const uint2 pb = o_part[r * 32 + lane];
+            const float b0 = __uint_as_float(pb.x << 16), b1 = __uint_as_float(pb.x & 0xFFFF0000u);
+            const float b2 = __uint_as_float(pb.y << 16), b3 = __uint_as_float(pb.y & 0xFFFF0000u);
+            const float inv = 1.f / tot;
+            a.x = (a.x * wa + b0 * wb) * inv;
+            a.y = (a.y * wa + b1 * wb) * inv;
+            a.z = (a.z * wa + b2 * wb) * inv;
+            a.w = (a.w * wa + b3 * wb) * inv;
+            lse = m + logf(tot);
+            reinterpret_cast<float4*>(o_acc)[r * 32 + lane] = a;
+            if (lane == 0) lse_acc[r] = lse;
+        }
+        if (out != nullptr) out[r * 32 + lane] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
     }
 }
 
@@ -993,16 +1056,19 @@ static DeviceInfo& device_info(int dev) {
         di.sms = sms;
         di.ok = (major == 10 && minor == 0) ? 1 : 0;
         if (di.ok &&
-            cudaFuncSetAttribute(hv_attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-                cudaSuccess)
+            (cudaFuncSetAttribute(hv_attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  SMEM_BYTES) != cudaSuccess ||
+             cudaFuncSetAttribute(hv_attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  SMEM_BYTES) != cudaSuccess))
             di.ok = 0;
         // The warpgroups' setmaxnreg split adds up to exactly 512 threads x 128
         // registers; a kernel launched with fewer would wait forever on the
         // increase, so refuse to launch one.
-        cudaFuncAttributes fa;
-        if (di.ok && (cudaFuncGetAttributes(&fa, hv_attn_fwd_kernel) != cudaSuccess ||
-                      fa.numRegs * NUM_THREADS < static_cast<int>(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE +
-                                                                  128 * REGS_CONTROL)))
+        const int split = static_cast<int>(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL);
+        cudaFuncAttributes fa, fb;
+        if (di.ok && (cudaFuncGetAttributes(&fa, hv_attn_fwd_kernel<false>) != cudaSuccess ||
+                      cudaFuncGetAttributes(&fb, hv_attn_fwd_kernel<true>) != cudaSuccess ||
+                      fa.numRegs * NUM_THREADS < split || fb.numRegs * NUM_THREADS < split))
             di.ok = 0;
     }
     return di;
@@ -1095,16 +1161,25 @@ static void* noalloc_scratch(int dev) {
     return addr[dev & 63];
 }
 
+// Row blocks of a ring-attention step (see Params); the standard call is the
+// whole sequence against itself.
+struct Blocks {
+    int Sk, q_vid, q_pos0, k_vid, k_pos0;
+    const int* kv_len;   // host, B entries, each in [1, Sk]
+    float* lse;          // device or nullptr
+};
+
 static int launch_attention(const Call& call, const void* q, const void* k, const void* v, void* out, int B,
                             int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
                             float scale, bool k_rotated, const float* qk_gamma, float qk_eps,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const Blocks* blk = nullptr) {
     (void)text_len;
     Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
     std::memset(prm, 0, sizeof(Params));
     const int S = call.S;
-    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, S, heads) ||
-        !make_qkv_map(&prm->tm_v, v, B, S, heads)) {
+    const int Sk = blk ? blk->Sk : S;
+    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, Sk, heads) ||
+        !make_qkv_map(&prm->tm_v, v, B, Sk, heads)) {
         delete prm;
         return HV_ERR_LAUNCH;
     }
@@ -1129,9 +1204,23 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->theta_log2 = static_cast<float>(std::log2(static_cast<double>(rope_theta)));
     prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     prm->timeout_ns = kWaitTimeoutNs;
-    for (int b = 0; b < B; ++b) prm->text_valid[b] = text_valid[b];
+    prm->Sk = Sk;
+    if (blk) {
+        prm->q_vid = blk->q_vid;
+        prm->q_pos0 = blk->q_pos0;
+        prm->k_vid = blk->k_vid;
+        prm->k_pos0 = blk->k_pos0;
+        prm->lse = blk->lse;
+        for (int b = 0; b < B; ++b) prm->kv_len[b] = blk->kv_len[b];
+    } else {
+        prm->q_vid = prm->k_vid = call.N;
+        for (int b = 0; b < B; ++b) prm->kv_len[b] = call.N + text_valid[b];
+    }
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
-    hv_attn_fwd_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    if (blk)
+        hv_attn_fwd_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    else
+        hv_attn_fwd_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     delete prm;
     const cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
@@ -1143,7 +1232,7 @@ static int launch_rope_k(const Call& call, const void* k, void* dst, int heads, 
                          const float* qk_gamma, float qk_eps, cudaStream_t stream) {
     const long long n_chunks = static_cast<long long>(call.bytes / 16);
     hv_rope_k_kernel<<<8 * call.sms, 256, 0, stream>>>(
-        static_cast<const uint4*>(k), static_cast<uint4*>(dst), n_chunks, heads, call.S, call.N, Hp, Wp,
+        static_cast<const uint4*>(k), static_cast<uint4*>(dst), n_chunks, heads, call.S, call.N, 0, Hp, Wp,
         static_cast<float>(std::log2(static_cast<double>(rope_theta))), qk_gamma ? qk_gamma + D : nullptr,
         qk_gamma ? qk_gamma + 3 * D : nullptr, qk_eps);
     return cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
@@ -1370,6 +1459,71 @@ int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_h
     // the caller's stream completes after the last copy out
     for (int slot = 0; slot < 2 && good; ++slot) good = cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
     return good ? HV_OK : HV_ERR_LAUNCH;
+}
+
+int hv_attn_forward_block(const void* q, const void* k, const void* v, void* out, float* lse, int B, int heads,
+                          int T, int Hp, int Wp, int Sq, int q_video, int q_pos0, int Sk, int k_video, int k_pos0,
+                          const int* kv_len, float rope_theta, float scale, void* cuda_stream) {
+    using namespace hv;
+    if (!q || !k || !v || !out || !kv_len) return HV_ERR_NULL_POINTER;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+    if ((mis & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return HV_ERR_MISALIGNED;
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH || Sq < 1 || Sk < 1)
+        return HV_ERR_BAD_SHAPE;
+    const long long n_video = static_cast<long long>(T) * Hp * Wp;
+    if (q_video < 0 || q_video > Sq || k_video < 0 || k_video > Sk || q_pos0 < 0 || k_pos0 < 0 ||
+        q_pos0 + static_cast<long long>(q_video) > n_video || k_pos0 + static_cast<long long>(k_video) > n_video)
+        return HV_ERR_BAD_SHAPE;
+    for (int b = 0; b < B; ++b)
+        if (kv_len[b] < 1 || kv_len[b] > Sk) return HV_ERR_BAD_TEXT;
+    if (!std::isfinite(rope_theta) || !(rope_theta > 0.f) || !std::isfinite(scale)) return HV_ERR_BAD_SCALAR;
+    const long long units = static_cast<long long>(B) * heads * ((Sq + UNIT_ROWS - 1) / UNIT_ROWS);
+    const long long big = static_cast<long long>(Sq > Sk ? Sq : Sk);
+    if (big + UNIT_ROWS >= (1ll << 31) || big * heads * D >= (1ll << 31) || units >= (1ll << 31) ||
+        n_video >= (1ll << 31))
+        return HV_ERR_TOO_LARGE;
+    const size_t qb = static_cast<size_t>(B) * Sq * heads * D * 2, kb = static_cast<size_t>(B) * Sk * heads * D * 2;
+    const size_t lb = static_cast<size_t>(B) * Sq * heads * 4;
+    if (ranges_overlap(out, qb, q, qb) || ranges_overlap(out, qb, k, kb) || ranges_overlap(out, qb, v, kb))
+        return HV_ERR_ALIAS;
+    if (lse && (ranges_overlap(lse, lb, out, qb) || ranges_overlap(lse, lb, q, qb) || ranges_overlap(lse, lb, k, kb) ||
+                ranges_overlap(lse, lb, v, kb)))
+        return HV_ERR_ALIAS;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    DeviceInfo& di = device_info(dev);
+    if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    Call call;
+    call.S = Sq;
+    call.N = static_cast<int>(n_video);
+    call.sms = di.sms;
+    call.units = units;
+    call.bytes = qb;
+    const Blocks blk{Sk, q_video, q_pos0, k_video, k_pos0, kv_len, lse};
+    return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, 0, nullptr, rope_theta, scale, false, nullptr,
+                            0.f, static_cast<cudaStream_t>(cuda_stream), &blk);
+}
+
+int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* out, long long rows,
+                  void* cuda_stream) {
+    using namespace hv;
+    if (!o_acc || !lse_acc || !o_part || !lse_part) return HV_ERR_NULL_POINTER;
+    if ((reinterpret_cast<uintptr_t>(o_acc) & 15u) || (reinterpret_cast<uintptr_t>(o_part) & 7u) ||
+        (reinterpret_cast<uintptr_t>(out) & 7u) || (reinterpret_cast<uintptr_t>(lse_acc) & 3u) ||
+        (reinterpret_cast<uintptr_t>(lse_part) & 3u))
+        return HV_ERR_MISALIGNED;
+    if (rows < 0) return HV_ERR_BAD_SHAPE;
+    if (rows == 0) return HV_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
+    DeviceInfo& di = device_info(dev);
+    if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    const long long blocks = (rows + 7) / 8;
+    const int grid = static_cast<int>(blocks < 16ll * di.sms ? blocks : 16ll * di.sms);
+    hv_merge_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+        o_acc, lse_acc, static_cast<const uint2*>(o_part), lse_part, static_cast<uint2*>(out), rows);
+    return cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
 int hv_attn_last_device_error(void) {

@@ -27,7 +27,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", "hv_attn_forward_qknorm",
             "hv_attn_forward_qknorm_ws", "hv_attn_forward_host", "hv_attn_host_workspace_bytes",
-            "hv_attn_workspace_bytes",
+            "hv_attn_workspace_bytes", "hv_attn_forward_block", "hv_attn_merge",
             "hv_video_tokens",
             "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
 
@@ -69,6 +69,11 @@ def lib() -> ctypes.CDLL:
             ctypes.c_size_t, ctypes.c_void_p]
         L.hv_attn_host_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_host_workspace_bytes.argtypes = [ctypes.c_int] * 7
+        L.hv_attn_forward_block.restype = ctypes.c_int
+        L.hv_attn_forward_block.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 11 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
+        L.hv_attn_merge.restype = ctypes.c_int
+        L.hv_attn_merge.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_longlong, ctypes.c_void_p]
         L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
@@ -241,6 +246,67 @@ def attn_forward_qknorm(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid,
     if st != HV_OK:
         raise HVError(st, "hv_attn_forward_qknorm_ws" if two_stage else "hv_attn_forward_qknorm")
     return out
+
+
+def attn_forward_block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, q_video: int, q_pos0: int,
+                       k_video: int, k_pos0: int, kv_len, rope_theta: float = 256.0, scale: float | None = None,
+                       out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                       stream: torch.cuda.Stream | None = None):
+    """One ring-attention step (``hv_attn_forward_block``): q [B, Sq, H, 128]
+    against k, v [B, Sk, H, 128]; returns (out bf16 [B, Sq, H, 128], lse fp32
+    [B, Sq, H])."""
+    _check(q, "q")
+    _check(k, "k")
+    _check(v, "v", k.shape)
+    if k.shape[0] != q.shape[0] or k.shape[2] != q.shape[2]:
+        raise ValueError("q and k/v must agree in batch and heads")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    b_sz, sq, heads, _ = q.shape
+    sk = k.shape[1]
+    if lse is None:
+        lse = torch.empty((b_sz, sq, heads), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (b_sz, sq, heads):
+        raise ValueError("lse must be contiguous float32 [B, Sq, heads]")
+    if len(kv_len) != b_sz:
+        raise ValueError("kv_len needs one entry per batch sample")
+    t_lat, hp, wp = (int(x) for x in grid)
+    kvl = (ctypes.c_int * b_sz)(*[int(x) for x in kv_len])
+    if scale is None:
+        scale = 1.0 / math.sqrt(128)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = lib().hv_attn_forward_block(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                         b_sz, heads, t_lat, hp, wp, sq, int(q_video), int(q_pos0), sk,
+                                         int(k_video), int(k_pos0), kvl, float(rope_theta), float(scale),
+                                         ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_forward_block")
+    return out, lse
+
+
+def attn_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, lse_part: torch.Tensor,
+               out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> None:
+    """``hv_attn_merge``: fold (o_part bf16, lse_part fp32) into (o_acc fp32, lse_acc fp32) in place;
+    optionally also write the merged rows to ``out`` (bf16)."""
+    rows = lse_acc.numel()
+    for name, t, dt in (("o_acc", o_acc, torch.float32), ("lse_acc", lse_acc, torch.float32),
+                        ("o_part", o_part, torch.bfloat16), ("lse_part", lse_part, torch.float32)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    if o_acc.numel() != rows * 128 or o_part.numel() != rows * 128 or lse_part.numel() != rows:
+        raise ValueError("o_acc / o_part must hold 128 channels per row of lse_acc; lse_part one per row")
+    if out is not None and (out.dtype != torch.bfloat16 or out.numel() != rows * 128 or not out.is_contiguous()):
+        raise ValueError("out must be contiguous bf16 with 128 channels per row")
+    if stream is None:
+        stream = torch.cuda.current_stream(o_acc.device)
+    with torch.cuda.device(o_acc.device):
+        st = lib().hv_attn_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                 None if out is None else out.data_ptr(), rows, ctypes.c_void_p(stream.cuda_stream))
+    if st != HV_OK:
+        raise HVError(st, "hv_attn_merge")
 
 
 def default_head_groups(heads: int) -> int:

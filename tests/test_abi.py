@@ -136,6 +136,30 @@ def test_host_entry_point_validates_arguments(lib):
     assert f(hq, hk, hv, ho, *args, 2, 0x900000, 1000, None) == 11            # too small
 
 
+def test_block_and_merge_entry_points_validate_arguments(lib):
+    kv = (ctypes.c_int * 1)(10)
+    f = lib.hv_attn_forward_block
+    q, k, v, o, lse = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    grid = (2, 4, 4)                                   # 32 video tokens
+    ok = (1, 2, *grid, 40, 20, 0, 16, 16, 8, kv, 256.0, 0.088, None)
+    assert f(None, k, v, o, lse, *ok) == 1
+    assert f(q, k, v, o, lse + 2, *ok) == 2                                       # lse misaligned
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 41, 0, 16, 16, 8, kv, 256.0, 0.088, None) == 3   # q_video > Sq
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 13, 16, 16, 8, kv, 256.0, 0.088, None) == 3  # past the grid
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 17, kv, 256.0, 0.088, None) == 3  # k past the grid
+    bad = (ctypes.c_int * 1)(17)
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, bad, 256.0, 0.088, None) == 4  # kv_len > Sk
+    zero = (ctypes.c_int * 1)(0)
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, zero, 256.0, 0.088, None) == 4
+    assert f(q, k, v, q + 64, lse, *ok) == 6                                      # out over q
+    assert f(q, k, v, o, o + 16, *ok) == 6                                        # lse over out
+    m = lib.hv_attn_merge
+    assert m(None, 0x10, 0x20, 0x30, None, 4, None) == 1
+    assert m(0x1008, 0x10, 0x20, 0x30, None, 4, None) == 2                        # o_acc not 16-byte aligned
+    assert m(0x1000, 0x10, 0x20, 0x30, None, -1, None) == 3
+    assert m(0x1000, 0x10, 0x20, 0x30, None, 0, None) == 0                        # nothing to merge
+
+
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
     import torch
     if torch.cuda.is_available():
