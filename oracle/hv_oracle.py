@@ -36,7 +36,7 @@ Sources (pages on HunyuanVideo; cited by page title and section):
 * [P4] README mirror (gittoolsai.com, Tencent-Hunyuan--HunyuanVideo),
   "单 GPU 推理": the supported height/width/frame settings.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
   R1 pairing: adjacent channel pairs (2i, 2i+1) inside each axis segment (the
      RoFormer rotation the pages cite in [P1] §5.5).
