@@ -57,18 +57,25 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v720x1280x129")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiling runs)")
     ap.add_argument("--no-ws", action="store_true", help="skip timing the workspace (pre-rotated K) path")
     ap.add_argument("--no-qknorm", action="store_true", help="skip timing the QK RMSNorm prologue paths")
+    ap.add_argument("--no-workloads", action="store_true", help="skip timing the other workloads")
     return ap.parse_args()
 
 
 def workload_flops(wl, text_valid) -> float:
     s_len = wl.seq_len
     return float(sum(4.0 * wl.heads * s_len * (wl.n_video + int(v)) * 128 for v in text_valid))
+
+
+def l2_note(wl) -> str:
+    gb = 4 * wl.batch * wl.seq_len * wl.heads * 256 / 1e9
+    if gb * 1e3 > 126:
+        return "inputs larger than L2 (q,k,v,out = %.2f GB vs 126 MB L2), no flush" % gb
+    return "inputs fit in L2 (q,k,v,out = %.1f MB vs 126 MB L2), no flush" % (gb * 1e3)
 
 
 def config_of(wl, text_valid) -> dict:
@@ -84,8 +91,7 @@ def config_of(wl, text_valid) -> dict:
         "text_valid": [int(v) for v in text_valid],
         "rope_theta": 256.0,
         "scale": 1.0 / math.sqrt(128),
-        "l2": "inputs larger than L2 (q,k,v,out = %.2f GB vs 126 MB L2), no flush" % (
-            4 * wl.batch * wl.seq_len * wl.heads * 256 / 1e9),
+        "l2": l2_note(wl),
         "parallelism": "replicas",
     }
 
@@ -211,67 +217,159 @@ def barrier(world: int):
         dist.barrier()
 
 
-def oracle_sample(wl, inp, seconds: float, seed: int = 0):
-    """Time the float64 oracle on sampled query rows of one (b, head): returns (tflops, info)."""
-    from threadpoolctl import threadpool_info
+def oracle_rows(wl) -> int:
+    """Rows per oracle sample: about 4e10 FLOP of float64 work against all valid keys (64..4096)."""
+    kv = wl.n_video + wl.text_len
+    return int(max(64, min(4096, round(4e10 / (4.0 * kv * 128)))))
+
+
+def oracle_estimate(wl, seed: int = 0, rows: int | None = None, threads: int | None = None) -> dict:
+    """Time the float64 oracle on one (b, head) of the workload and extrapolate to the whole call.
+
+    The oracle rotates a head's keys once and then computes each query row
+    against all valid keys, so its time for r rows of one head is a + b*r. Two
+    calls of ``joint_attention_head`` (32 rows, then 32 + ``rows`` rows) give a
+    (key preparation) and b (per row); the whole call takes B*heads*(a + b*S).
+    Inputs: one head's q, k, v of the workload's shape from the seeded
+    generator (the oracle's time does not depend on the values).
+    ``threads``: limit of the BLAS thread pools (None: all).
+    """
+    from threadpoolctl import threadpool_info, threadpool_limits
 
     from joint_full_attention_b200 import workloads as W
     from oracle import hv_oracle as O
 
-    b, h = 0, 0
-    valid = int(inp["text_valid"][b])
-    q = W.bf16_bits_to_f64(inp["q"][b:b + 1, :, h:h + 1])
-    k = W.bf16_bits_to_f64(inp["k"][b:b + 1, :, h:h + 1])
-    v = W.bf16_bits_to_f64(inp["v"][b:b + 1, :, h:h + 1])
+    one = W.Workload(wl.name + "-head", wl.label, 1, 1, wl.grid, wl.text_len, valid=wl.valid,
+                     k_head_scale=False)
+    inp = W.make_inputs(one, seed=seed)
+    valid = int(inp["text_valid"][0])
+    q, k, v = (W.bf16_bits_to_f64(inp[n][0, :, 0]) for n in ("q", "k", "v"))
+    rows = oracle_rows(wl) if rows is None else int(rows)
     rng = np.random.default_rng(seed)
-    kv = wl.n_video + valid
 
-    def run(rows):
-        samples = np.stack([np.zeros(rows, np.int64), np.zeros(rows, np.int64),
-                            rng.integers(0, wl.seq_len, rows)], axis=1)
+    def run(r):
+        sel = rng.integers(0, wl.seq_len, r)
         t0 = time.perf_counter()
-        O.joint_attention_samples(q, k, v, wl.grid, wl.text_len, [valid], samples)
+        O.joint_attention_head(q, k, v, wl.grid, valid, rows=sel)
         return time.perf_counter() - t0
 
-    rows = 32
-    dt = run(rows)
-    rows = int(max(32, min(1 << 16, rows * seconds / max(dt, 1e-3) * 0.8)))
-    dt = run(rows)
-    flops = 4.0 * rows * kv * 128
-    threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
-    info = {"rows": rows, "seconds": dt, "threads": threads,
-            "sample": f"{rows} query rows of (b=0, head=0) against all {kv} valid keys, "
-                      f"float64 numpy oracle incl. the per-head key rotation; TFLOP/s of the sampled rows"}
-    return flops / dt / 1e12, info
+    with threadpool_limits(limits=threads):
+        used = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+        t_all = time.perf_counter()
+        run(1)                                  # warm-up: first-touch and allocation effects
+        t1 = min(run(32), run(32))
+        t2 = run(32 + rows)
+        t_all = time.perf_counter() - t_all
+    per_row = max((t2 - t1) / rows, 1e-9)
+    fixed = max(t1 - 32 * per_row, 0.0)
+    call_s = wl.batch * wl.heads * (fixed + per_row * wl.seq_len)
+    return {"call_seconds": call_s, "per_row_s": per_row, "per_head_fixed_s": fixed, "rows": rows,
+            "threads": used, "sample_seconds": t_all,
+            "sample": f"float64 oracle (joint_attention_head) on one (b, head) of this workload, all valid "
+                      f"keys: after a warm-up call, 32 seeded query rows (best of 2) and {32 + rows} rows; "
+                      f"time = a + b*rows fitted (a: the head's key rotation, b: per row), extrapolated to "
+                      f"B*heads*(a + b*S)"}
 
 
-def run_reference(args, wl, inp, rank, world):
+def cpu_baseline_of(wl, flops: float, seed: int = 0, one_core: bool = True) -> dict:
+    """The oracle on all host threads (and on one core), extrapolated to the whole call."""
+    full = oracle_estimate(wl, seed)
+    res = {"value": flops / full["call_seconds"] / 1e12, "unit": UNIT, "cores": full["threads"],
+           "kind": "oracle", "sample": full["sample"],
+           "rows": full["rows"], "ms_per_call_extrapolated": full["call_seconds"] * 1e3,
+           "cpu_seconds": full["sample_seconds"], "host_cpus": os.cpu_count()}
+    if one_core:
+        one = oracle_estimate(wl, seed, rows=max(16, full["rows"] // 4), threads=1)
+        res["one_core"] = {"value": flops / one["call_seconds"] / 1e12, "cores": 1, "rows": one["rows"],
+                           "ms_per_call_extrapolated": one["call_seconds"] * 1e3,
+                           "cpu_seconds": one["sample_seconds"]}
+    return res
+
+
+def run_reference(args, wl, rank, world):
     if rank != 0:
         return
-    cfg = config_of(wl, inp["text_valid"])
-    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.warmup):
-        oracle_sample(wl, inp, min(per_step, 2.0))
-    vals, infos = [], []
+    from joint_full_attention_b200 import workloads as W
+    text_valid = W.text_valid_of(wl, seed=0)
+    cfg = config_of(wl, text_valid)
+    flops = workload_flops(wl, text_valid)
+    for w in range(args.warmup):
+        oracle_estimate(wl, seed=100 + w, rows=32)
+    calls = []
     t_all = time.perf_counter()
     for s in range(args.steps):
-        v, info = oracle_sample(wl, inp, per_step, seed=s + 1)
-        vals.append(v)
-        infos.append(info)
+        calls.append(oracle_estimate(wl, seed=s + 1))
     wall = time.perf_counter() - t_all
-    value = statistics.mean(vals)
-    flops = workload_flops(wl, inp["text_valid"])
-    ms = flops / (value * 1e12) * 1e3
+    call_s = statistics.mean(c["call_seconds"] for c in calls)
+    value = flops / call_s / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": call_s * 1e3,
+        "ms_per_step_extrapolated": True, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": infos[-1]["threads"], "kind": "oracle",
-                         "sample": infos[-1]["sample"] + f"; {args.steps} steps in {wall:.1f} s, "
-                                   f"ms_per_step extrapolated to the full call"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": calls[-1]["threads"], "kind": "oracle",
+                         "rows": calls[-1]["rows"],
+                         "sample": calls[-1]["sample"] + f"; each step is one such estimate, {args.steps} "
+                                   f"steps in {wall:.1f} s; ms_per_step is the extrapolated whole call, "
+                                   f"not a measured call"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def time_calls(call, stream, steps: int, warmup: int) -> list[float]:
+    """CUDA-event device time (ms) of each of `steps` calls after `warmup` untimed ones."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def other_workloads(args, dev, stream, peaks):
+    """Device time, TFLOP/s and roofline fraction of the fused call on every other workload."""
+    import torch
+
+    from joint_full_attention_b200 import hvattn as H
+    from joint_full_attention_b200 import workloads as W
+
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    res = []
+    for name, wl in W.WORKLOADS.items():
+        if name == args.workload:
+            continue
+        inp = W.make_device_inputs(wl, seed=0, device=dev)
+        tv = [int(x) for x in inp["text_valid"]]
+        out = torch.empty_like(inp["q"])
+        flops = workload_flops(wl, tv)
+        call = lambda: H.attn_forward(inp["q"], inp["k"], inp["v"], wl.grid, wl.text_len, tv, out=out,
+                                      stream=stream)
+        one = statistics.median(time_calls(call, stream, 3, 2))
+        steps = int(max(5, min(200, 1500.0 / max(one, 1e-3))))
+        ms = time_calls(call, stream, steps, 2)
+        if H.last_device_error() != 0:
+            raise RuntimeError(f"device error on workload {name}")
+        mean = statistics.mean(ms)
+        achieved = flops / (mean / 1e3) / 1e12
+        entry = {"workload": name, "label": wl.label, "batch": wl.batch, "heads": wl.heads, "grid": list(wl.grid),
+                 "seq_len": wl.seq_len, "text_valid": tv, "flop_per_call": flops, "steps": steps,
+                 "ms_per_call": mean, "ms_min": min(ms), "value": achieved, "unit": UNIT,
+                 "frac_of_sustained": achieved / peak, "frac_of_burst": achieved / peak_burst,
+                 "units_512_rows": wl.batch * wl.heads * -(-wl.seq_len // 512), "sms": sms}
+        if not args.no_cpu_baseline:
+            entry["cpu_baseline"] = cpu_baseline_of(wl, flops, one_core=False)
+        res.append(entry)
+        del inp, out
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args, wl, inp, rank, world, local):
@@ -389,10 +487,17 @@ def run_ours(args, wl, inp, rank, world, local):
         e2e_ms, e2e_value = replica_throughput(e0.elapsed_time(e1) / args.e2e_steps, flops, world)
         e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * qh.numel() * 2,
                "d2h_bytes_per_step": oh.numel() * 2, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
+        del qh, kh, vh, oh, work
+
+    peaks, peak_kind = load_peaks()
+    others = None
+    if not args.no_workloads:
+        del q, k, v, out
+        torch.cuda.empty_cache()
+        others = other_workloads(args, dev, stream, peaks)
 
     if rank != 0:
         return
-    peaks, peak_kind = load_peaks()
     mean_launch = statistics.mean(launch_ms)
     achieved = flops / (mean_launch / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -416,11 +521,10 @@ def run_ours(args, wl, inp, rank, world, local):
         "clocks": clk,
         "workspace_path": ws_line,
         "qk_norm_path": qk_line,
+        "workloads": others,
     }
     if world == 1 and not args.no_cpu_baseline:
-        cpu_value, info = oracle_sample(wl, inp, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": cpu_value, "unit": UNIT, "cores": info["threads"], "kind": "oracle",
-                                "sample": info["sample"]}
+        line["cpu_baseline"] = cpu_baseline_of(wl, flops)
     print(json.dumps(line), flush=True)
 
 
@@ -433,7 +537,7 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))
         if rank == 0:
-            run_reference(args, wl, W.make_inputs(wl, seed=0), rank, world)
+            run_reference(args, wl, rank, world)
         return
     rank, world, local = dist_init(args.gpus)
     inp = W.make_inputs(wl, seed=0)

@@ -176,9 +176,10 @@ long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int t
  * hv_attn_forward. Problems needing more than HV_NOALLOC_MAX_BYTES of
  * rotated keys (B * S * heads * 256 bytes) are rejected with
  * HV_ERR_NOALLOC_LIMIT before anything is launched. It calls no cudaMalloc,
- * cudaFree or other allocating routine. The first call on a device looks up
- * the scratch array's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture. Every call on a
+ * cudaFree or other allocating routine. Every call looks up the scratch
+ * array's device address in the current context (cudaGetSymbolAddress); the
+ * first call on a device also loads the library's kernels there, so make it
+ * before any stream capture. Every call on a
  * device shares the one scratch array, which keeps the last call's contents:
  * calls whose kernels overlap on the GPU (different streams, or different
  * host threads) race on it and must be ordered by the caller.

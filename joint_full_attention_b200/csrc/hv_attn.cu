@@ -1146,19 +1146,15 @@ static int validate(const void* q, const void* k, const void* v, const void* out
 // allocation call ever creates it. All calls share it.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[HV_NOALLOC_MAX_BYTES];
 
-// Device address of g_noalloc_scratch on device `dev` (which must be the
-// current device), looked up once per device and then cached. In host code
-// the array's name is only a stand-in; the address must come from the runtime.
-static void* noalloc_scratch(int dev) {
-    static void* addr[64] = {};
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev & 63]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        addr[dev & 63] = ptr;
-    }
-    return addr[dev & 63];
+// Device address of g_noalloc_scratch in the current context. In host code
+// the array's name is only a stand-in; the address must come from the
+// runtime. It is looked up on every call (a cheap table lookup once the
+// module is loaded), so a context that was reset and re-created, where the
+// array may sit elsewhere, never sees a stale address.
+static void* noalloc_scratch() {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    return ptr;
 }
 
 // Row blocks of a ring-attention step (see Params); the standard call is the
@@ -1379,9 +1375,7 @@ int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* o
     int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call);
     if (st != HV_OK) return st;
     if (call.bytes > HV_NOALLOC_MAX_BYTES) return HV_ERR_NOALLOC_LIMIT;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
-    void* scratch = noalloc_scratch(dev);
+    void* scratch = noalloc_scratch();
     if (!scratch) return HV_ERR_LAUNCH;
     // the first stage overwrites every byte of the scratch it uses, so
     // nothing left there by an earlier call needs clearing

@@ -101,14 +101,12 @@ def _normal_bf16(rng: np.random.Generator, shape, head_scale: np.ndarray | None 
     return out
 
 
-def make_inputs(wl: Workload, seed: int = 0) -> dict:
-    """Seeded inputs of a workload.
-
-    Returns dict with q, k, v as uint16 bf16 bit arrays [B, S, heads, 128],
-    text_valid (int32 [B]) and k_scale (float32 [heads] or None).
-    """
+def _streams(wl: Workload, seed: int):
     root = np.random.SeedSequence([seed, sum(map(ord, wl.name))])
-    s_meta, s_q, s_k, s_v = root.spawn(4)
+    return root.spawn(4)
+
+
+def _meta(wl: Workload, s_meta) -> tuple[np.ndarray, np.ndarray | None]:
     meta = np.random.Generator(np.random.PCG64(s_meta))
     if wl.valid is not None:
         text_valid = np.asarray(wl.valid, dtype=np.int32)
@@ -116,6 +114,45 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
         text_valid = meta.integers(20, 257, size=wl.batch).astype(np.int32)
     text_valid = np.minimum(text_valid, wl.text_len).astype(np.int32)
     k_scale = meta.uniform(0.5, 2.0, size=wl.heads).astype(np.float32) if wl.k_head_scale else None
+    return text_valid, k_scale
+
+
+def text_valid_of(wl: Workload, seed: int = 0) -> np.ndarray:
+    """The valid text lengths ``make_inputs(wl, seed)`` draws, without drawing the tensors."""
+    return _meta(wl, _streams(wl, seed)[0])[0]
+
+
+def make_device_inputs(wl: Workload, seed: int, device) -> dict:
+    """Inputs of the workload's shape and distribution drawn on the GPU (torch's seeded
+    Philox generator): for timing runs, where drawing 100+ million values on the host
+    would dominate. Same recipe as ``make_inputs`` (N(0, 1) in float32, K scaled per
+    head when the workload asks for it, rounded to bf16); not the same values.
+    """
+    import torch
+
+    text_valid, k_scale = _meta(wl, _streams(wl, seed)[0])
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) * 1000003 + sum(map(ord, wl.name)))
+    shape = (wl.batch, wl.seq_len, wl.heads, HEAD_DIM)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+        if name == "k" and k_scale is not None:
+            x *= torch.from_numpy(k_scale).to(device).view(1, 1, -1, 1)
+        out[name] = x.to(torch.bfloat16)
+        del x
+    out["text_valid"] = text_valid
+    return out
+
+
+def make_inputs(wl: Workload, seed: int = 0) -> dict:
+    """Seeded inputs of a workload.
+
+    Returns dict with q, k, v as uint16 bf16 bit arrays [B, S, heads, 128],
+    text_valid (int32 [B]) and k_scale (float32 [heads] or None).
+    """
+    s_meta, s_q, s_k, s_v = _streams(wl, seed)
+    text_valid, k_scale = _meta(wl, s_meta)
     shape = (wl.batch, wl.seq_len, wl.heads, HEAD_DIM)
     q = _normal_bf16(np.random.Generator(np.random.PCG64(s_q)), shape)
     k = _normal_bf16(np.random.Generator(np.random.PCG64(s_k)), shape, head_scale=k_scale)
