@@ -81,7 +81,14 @@ enum hv_status {
  * synchronising. Errors in the arguments are reported before anything is
  * launched. A kernel-side wait that runs out (a broken pipeline, never an
  * expected event) sets the device error word read by
- * hv_attn_last_device_error; the kernel then ends cleanly.
+ * hv_attn_last_device_error and a status word in host memory; the kernel then
+ * ends cleanly. While that status word is set, every entry point that
+ * launches work on the device returns HV_ERR_DEVICE_TIMEOUT without
+ * launching (checked without synchronising), until hv_attn_last_device_error
+ * reads and clears it. The status words live in one static 4 KB page of host
+ * memory that the first call on a device page-locks and maps for the device
+ * (cudaHostRegister: a registration, not an allocation); make that first call
+ * before any stream capture.
  */
 int hv_attn_forward(const void* q, const void* k, const void* v, void* out,
                     int B, int heads, int T, int Hp, int Wp,
@@ -245,7 +252,10 @@ long long hv_attn_host_workspace_bytes(int B, int heads, int T, int Hp, int Wp, 
  * the 3D RoPE of those tokens; the remaining rows are text (not rotated).
  * Only the first kv_len[b] key rows of sample b take part.
  *
- * q, out   : device bf16 [B, Sq, heads, 128]; k, v: device bf16 [B, Sk, heads, 128].
+ * q        : device bf16 [B, Sq, heads, 128]; k, v: device bf16 [B, Sk, heads, 128].
+ * out      : device [B, Sq, heads, 128], bf16 (out_fp32 = 0) or fp32 (out_fp32 = 1:
+ *            the block's partial result kept at full precision for hv_attn_merge,
+ *            so that a long ring adds no bf16 rounding per step).
  * lse      : device fp32 [B, Sq, heads] or NULL; lse = log(sum_j exp(s_j)) of
  *            the scaled scores s_j = scale * q'.k'_j over the block's keys.
  * kv_len   : HOST pointer to B ints, 1 <= kv_len[b] <= Sk (a block with no
@@ -260,22 +270,25 @@ long long hv_attn_host_workspace_bytes(int B, int heads, int T, int Hp, int Wp, 
 int hv_attn_forward_block(const void* q, const void* k, const void* v, void* out, float* lse,
                           int B, int heads, int T, int Hp, int Wp,
                           int Sq, int q_video, int q_pos0, int Sk, int k_video, int k_pos0,
-                          const int* kv_len, float rope_theta, float scale, void* cuda_stream);
+                          const int* kv_len, float rope_theta, float scale, int out_fp32,
+                          void* cuda_stream);
 
 /*
- * hv_attn_merge - fold one key block's result (o_part bf16, lse_part fp32)
- * into the running result (o_acc fp32, lse_acc fp32) of the same `rows` query
- * rows of 128 channels: with m = max(lse_acc, lse_part), w = exp(lse - m),
+ * hv_attn_merge - fold one key block's result (o_part, fp32 if o_part_fp32 = 1
+ * else bf16; lse_part fp32) into the running result (o_acc fp32, lse_acc fp32)
+ * of the same `rows` query rows of 128 channels: with m = max(lse_acc,
+ * lse_part), w = exp(lse - m),
  *   o_acc <- (w_acc o_acc + w_part o_part) / (w_acc + w_part),
  *   lse_acc <- m + log(w_acc + w_part),
  * the softmax over the union of the keys. Start from o_acc = 0 and
  * lse_acc = -inf. If `out` is not NULL the merged rows are also written to it
- * as bf16 (the last merge of a ring). Device pointers; o_acc 16-byte, o_part and
- * out 8-byte, lse 4-byte aligned. Asynchronous on cuda_stream. No
- * counterpart in the pages beyond the merge rule of ring attention.
+ * as bf16 (the last merge of a ring). Device pointers; o_acc 16-byte, o_part
+ * 16-byte (fp32) or 8-byte (bf16), out 8-byte, lse 4-byte aligned.
+ * Asynchronous on cuda_stream. No counterpart in the pages beyond the merge
+ * rule of ring attention.
  */
-int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* out,
-                  long long rows, void* cuda_stream);
+int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, int o_part_fp32, const float* lse_part,
+                  void* out, long long rows, void* cuda_stream);
 
 /*
  * hv_video_tokens - number of video tokens N = (floor((F-1)/4)+1)*(H/16)*(W/16)
@@ -288,9 +301,11 @@ long long hv_video_tokens(int frames, int height, int width);
 /*
  * hv_attn_last_device_error - synchronises the current device, returns the
  * device-side error word accumulated by kernels of this library since the
- * previous call, and clears it. 0 = none. Otherwise bit 0 is set for a wait
- * that ran out, and bits 8..15 name the waiting role (1 producer, 2 MMA,
- * 3 softmax, 4 RoPE, 5 self-test). Returns -1 if the device cannot be read.
+ * previous call, and clears it together with the device's host status word
+ * (after which the entry points launch again). 0 = none. Otherwise bit 0 is
+ * set for a wait that ran out, and bits 8..15 name the waiting role
+ * (1 producer, 2 MMA, 3 softmax, 4 RoPE, 5 self-test; several roles OR
+ * together). Returns -1 if the device cannot be read.
  */
 int hv_attn_last_device_error(void);
 
@@ -302,6 +317,25 @@ int hv_attn_last_device_error(void);
  * or hanging the GPU. Returns -1 on a CUDA error.
  */
 int hv_attn_selftest_timeout(int timeout_us);
+
+/*
+ * hv_attn_selftest_abort - a test of the attention kernel's own abort path,
+ * without faulting or hanging anything: runs hv_attn_forward's kernel (keys
+ * rotated on load, rope_theta 256, scale 1/sqrt(128)) on the caller's problem
+ * with every wait bounded by timeout_us microseconds (1000..1000000) and with
+ * CTA 0 leaving its K tile load number withhold_k (>= 0, counted over that
+ * CTA's loads) unissued, so that the wait of its RoPE warps for those keys
+ * runs out. That CTA then stops every role, lets its copies and MMAs in
+ * flight finish, frees its TMEM and returns, while the other CTAs finish. Synchronises `cuda_stream`, then returns HV_OK;
+ * the error word and the host status word are set as for any timeout (read
+ * and clear them with hv_attn_last_device_error). `out` is left partly
+ * written. Arguments as hv_attn_forward; HV_ERR_BAD_SCALAR for a bad
+ * withhold_k or timeout_us.
+ */
+int hv_attn_selftest_abort(const void* q, const void* k, const void* v, void* out,
+                           int B, int heads, int T, int Hp, int Wp,
+                           int text_len, const int* text_valid, int withhold_k, int timeout_us,
+                           void* cuda_stream);
 
 /* Static string for an hv_status code. */
 const char* hv_attn_status_string(int status);

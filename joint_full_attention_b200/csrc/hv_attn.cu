@@ -22,10 +22,16 @@
 // bf16 probabilities P_i overwrite the first 64 columns of S_i and feed the
 // PV MMA straight from TMEM.
 //
+// The two softmax warpgroups take turns for their exponentials (an mbarrier
+// hand-off per K tile): the MUFU unit of each SM sub-partition then serves one
+// warpgroup at a time at its full rate, which keeps each Q tile's chain
+// (softmax, then PV and the next QK on the tensor core) short while the other
+// tile's MMAs run.
+//
 // Every mbarrier wait is bounded by a %globaltimer budget; when one runs out
-// the CTA records the role in a device error word, tells the other roles to
-// stop, waits (bounded) for its own copies and MMAs in flight, frees its TMEM
-// and returns.
+// the CTA records the role in a device error word and in a host-visible status
+// word, tells the other roles to stop, waits (bounded) for its own copies and
+// MMAs in flight, frees its TMEM and returns.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -105,7 +111,8 @@ constexpr int B_V_EMPTY = B_V_FULL + VSTAGES_MAX;
 constexpr int B_S_FULL = B_V_EMPTY + VSTAGES_MAX;
 constexpr int B_P_READY = B_S_FULL + QTILES;
 constexpr int B_O_DONE = B_P_READY + QTILES;
-constexpr int B_DRAIN = B_O_DONE + QTILES;
+constexpr int B_TURN = B_O_DONE + QTILES;    // softmax warpgroup i may start its exponentials
+constexpr int B_DRAIN = B_TURN + QTILES;
 constexpr int NUM_BARS = B_DRAIN + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
@@ -128,7 +135,7 @@ struct __align__(64) Params {
     CUtensorMap tm_q;
     CUtensorMap tm_k;
     CUtensorMap tm_v;
-    __nv_bfloat16* out;
+    void* out;          // bf16 [B, S, H, 128], or fp32 when out_f32
     int B, H, S, N, T, Hp, Wp, HpWp;
     int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
     int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
@@ -142,6 +149,12 @@ struct __align__(64) Params {
     float theta_log2;   // log2(rope_theta)
     float scale_log2;   // scale * log2(e)
     unsigned long long timeout_ns;
+    unsigned int* status;   // host-visible status word (mapped pinned memory) or nullptr
+    int withhold_k;     // test hook: CTA 0 skips its K load number withhold_k (-1: off)
+    // place of this launch's heads in the whole call (a call split into head
+    // groups launches heads h_offset .. h_offset + H - 1 of h_total), and the
+    // round width of the traversal-direction rule (the device's SM count)
+    int h_total, h_offset, round_width;
     // Geometry of the row blocks. The standard call: Q and K/V are the whole
     // joint sequence (Sk = S, q_vid = k_vid = N, offsets 0). A ring-attention
     // block: Q rows and K/V rows are runs of the joint sequence whose first
@@ -149,6 +162,7 @@ struct __align__(64) Params {
     // at q_pos0 / k_pos0; the other rows are text.
     int Sk;             // rows of the K and V tensors (S: rows of Q and out)
     int q_vid, q_pos0, k_vid, k_pos0;
+    int out_f32;        // 1: out rows are fp32 (ring-attention partial results)
     float* lse;         // optional [B, S, H] fp32: natural-log log-sum-exp of each row's scaled scores
     int kv_len[HV_MAX_BATCH];   // keys taking part, per batch sample (the rest are masked)
 };
@@ -158,6 +172,19 @@ __device__ unsigned int g_dev_error = 0;
 struct Waiter {
     volatile int* abort_flag;
     unsigned long long timeout_ns;
+    unsigned int* status;
+    bool record = true;   // false for the bounded drains of an abort already recorded
+
+    // Record a wait that ran out in the error words, and stop every role of
+    // the CTA at its next wait.
+    __device__ __forceinline__ void fail(uint32_t role) const {
+        *abort_flag = 1;
+        if (!record) return;
+        const uint32_t word = 1u | (role << 8);
+        atomicOr(&g_dev_error, word);
+        if (status != nullptr) st_sys_u32(status, word);
+        __threadfence_block();
+    }
 
     // Spin until the phase of `bar` with `parity` has completed. Returns false
     // when the CTA is aborting (this wait ran out, or another role's did).
@@ -168,9 +195,7 @@ struct Waiter {
             if (mbar_try_wait(bar, parity)) return true;
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > timeout_ns) {
-                *abort_flag = 1;
-                atomicOr(&g_dev_error, 1u | (role << 8));
-                __threadfence_block();
+                fail(role);
                 return false;
             }
         }
@@ -200,8 +225,18 @@ struct Ring {
 
 struct UnitCoord {
     int b, h, qu, nt, last_lim;
+    int rev;   // 1: this unit walks the K/V tiles from the last to the first
+    // K/V tile visited at step j of the unit's loop
+    __device__ __forceinline__ int tile(int j) const { return rev ? nt - 1 - j : j; }
 };
 
+// Units are dealt to the CTAs round-robin, head-major, so the CTAs of one
+// round share a head's K/V through L2. Consecutive rounds walk the K/V tiles
+// in opposite directions: a CTA starting its next unit begins on the tiles it
+// (and the rest of the round) read last, which are still in L2. The
+// direction is a function of the unit's place in the whole call (its global
+// unit number over a fixed round width), so a call split into launches over
+// head groups sums in the same order and gives the same bits.
 __device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
     UnitCoord c;
     c.qu = u % p.n_qunits;
@@ -211,11 +246,15 @@ __device__ __forceinline__ UnitCoord decode_unit(const Params& p, int u) {
     const int kv_len = p.kv_len[c.b];
     c.nt = (kv_len + BN - 1) / BN;
     c.last_lim = kv_len - (c.nt - 1) * BN;
+    // < B * heads * ceil(S / 256) <= 2^24 (S * heads * 128 < 2^31, B <= 512): fits an int
+    const int ug = (c.b * p.h_total + p.h_offset + c.h) * p.n_qunits + c.qu;
+    c.rev = (ug / p.round_width) & 1;
     return c;
 }
 
-// Rotate the video rows (sequence index < N) of one 128-row tile in place.
-// Thread `rt` (0..127) owns 16-byte chunk cc = rt % 16 of rows rt/16 + 8k.
+// Rotate the video rows (sequence index < N) of one tile of ROWS rows (two
+// boxes of 64 channels) in place.
+// Thread `rt` (0..191) owns 16-byte chunk cc = rt % 16 of rows rt/16 + 12k.
 // A chunk holds channels [8cc, 8cc+8): four adjacent pairs, all inside one
 // axis segment because the segment borders 16 and 72 are multiples of 8.
 // Axis t: channels [0,16), 8 pairs; h: [16,72), 28 pairs; w: [72,128), 28 pairs.
@@ -346,20 +385,21 @@ __device__ __forceinline__ void advance8(GridPos& g, const Params& p) {
     }
 }
 
-// Rows n0 + rb, n0 + rb + 12, ... of a tile; local rows below `vid` are video
-// tokens whose global token index is pos0 + row (the rest are text, left as
-// they are).
+// Rows n0 + rb, n0 + rb + 12, ... of a tile of ROWS rows; sequence rows
+// below `vid` are video tokens whose global token index is pos0 + row (the
+// rest are text, left as they are).
+template <int ROWS>
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int vid, int pos0, int rt,
                                           const RopeLane& L, const Params& p) {
     const int rb = rt >> 4;
     int n = n0 + rb;
-    if (n >= vid) return;
+    if (n >= vid || rb >= ROWS) return;
     GridPos g;
     g.w = (pos0 + n) % p.Wp;
     const int th = (pos0 + n) / p.Wp;
     g.h = th % p.Hp;
     g.t = th / p.Hp;
-    const uint32_t box_base = tile + L.box * BOX_BYTES;
+    const uint32_t box_base = tile + L.box * (ROWS * 128);
     auto row_addr = [&](int r) { return box_base + r * 128 + ((L.cin ^ (r & 7)) << 4); };
     const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
@@ -367,9 +407,9 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
     if (p.use_table) {
         // two rows (r, r + ROPE_GROUPS) per iteration so that their loads overlap
 #pragma unroll 1
-        for (int r = rb; r < BM; r += 2 * ROPE_GROUPS) {
+        for (int r = rb; r < ROWS; r += 2 * ROPE_GROUPS) {
             const int pos0 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
-            const bool has1 = n + ROPE_GROUPS < vid && r + ROPE_GROUPS < BM;
+            const bool has1 = n + ROPE_GROUPS < vid && r + ROPE_GROUPS < ROWS;
             advance8(g, p);
             const int pos1 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
             const uint32_t a0 = row_addr(r);
@@ -394,7 +434,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
         }
     } else {
 #pragma unroll 1
-        for (int r = rb; r < BM; r += ROPE_GROUPS) {
+        for (int r = rb; r < ROWS; r += ROPE_GROUPS) {
             const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
             const uint32_t a = row_addr(r);
             uint4 d = lds128(a);
@@ -414,15 +454,17 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 }
 
 // RMSNorm prologue, then the rotation of the video rows, for every row of a
-// tile (rows rb, rb + 12, ...); text rows and rows past the sequence are only
-// normalised (rows past the sequence hold TMA's zero fill and stay zero).
-// gamma_v / gamma_t: shared-memory addresses of the video / text gamma of
-// this tensor (Q or K). Every lane of a warp runs the same number of
-// iterations (rb and rb + 1 share a warp and a trip count), as the row sum is
-// a half-warp shuffle.
+// tile of ROWS rows (rows rb, rb + 12, ...); text rows and rows past the
+// sequence are only normalised (rows past the sequence hold TMA's zero fill
+// and stay zero). gamma_v / gamma_t: shared-memory addresses of the video /
+// text gamma of this tensor (Q or K). Every lane of a warp runs the same
+// number of iterations (rb and rb + 1 share a warp, and as ROWS is even they
+// share a trip count), as the row sum is a half-warp shuffle.
+template <int ROWS>
 __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
                                                int n0, int vid, int pos0, int rt, const RopeLane& L,
                                                const Params& p) {
+    static_assert(ROWS % 2 == 0, "half-warp row pairs");
     const int rb = rt >> 4;
     int n = n0 + rb;
     GridPos g;
@@ -430,13 +472,13 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
     const int th = (pos0 + n) / p.Wp;
     g.h = th % p.Hp;
     g.t = th / p.Hp;
-    const uint32_t box_base = tile + L.box * BOX_BYTES;
+    const uint32_t box_base = tile + L.box * (ROWS * 128);
     const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
     const int stride = 2 * L.half_dim;
     const uint32_t gofs = 4u * static_cast<uint32_t>(L.ch0);
 #pragma unroll 1
-    for (int r = rb; r < BM; r += ROPE_GROUPS) {
+    for (int r = rb; r < ROWS; r += ROPE_GROUPS) {
         const bool video = n < vid;
         const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
         const uint32_t a = box_base + r * 128 + ((L.cin ^ (r & 7)) << 4);
@@ -500,9 +542,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
             if (p.qk_norm)
-                rope_norm_tile(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, q_vid, q_pos0, rt, L, p);
+                rope_norm_tile<BM>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, q_vid, q_pos0, rt, L,
+                                   p);
             else
-                rope_tile(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
+                rope_tile<BM>(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -511,11 +554,12 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
         for (int j = 0; j < c.nt; ++j, kr.next()) {
             if (!(ok = waiter.wait_warp(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
+            const int k0 = c.tile(j) * BN;
             if (p.qk_norm)
-                rope_norm_tile(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, j * BN, k_vid, k_pos0,
-                               rt, L, p);
-            else if (j * BN < k_vid)
-                rope_tile(sK + kr.s * TILE_BYTES, sTable, j * BN, k_vid, k_pos0, rt, L, p);
+                rope_norm_tile<BN>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, k0, k_vid,
+                                   k_pos0, rt, L, p);
+            else if (k0 < k_vid)
+                rope_tile<BN>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
@@ -547,8 +591,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 }
 
 // BLOCK: a ring-attention block (Q and K/V rows at their own global offsets,
-// log-sum-exp output); the standard call is compiled without that
-// generality (video rows = the first N rows of both, no offsets).
+// log-sum-exp and optionally fp32 output); the standard call is compiled
+// without that generality (video rows = the first N rows of both, no offsets).
 template <bool BLOCK>
 __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -581,6 +625,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             mbar_init(bar(B_S_FULL + i), 1);
             mbar_init(bar(B_P_READY + i), 4);
             mbar_init(bar(B_O_DONE + i), 1);
+            mbar_init(bar(B_TURN + i), 4);
         }
         mbar_init(bar(B_DRAIN), 1);
         *abort_flag = 0;
@@ -600,7 +645,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const Waiter waiter{abort_flag, p.timeout_ns};
+    const Waiter waiter{abort_flag, p.timeout_ns, p.status};
     const uint32_t sQ = base + OFF_Q;
     const uint32_t sK = base + OFF_KV;
     const uint32_t sV = sK + static_cast<uint32_t>(p.kstages) * TILE_BYTES;
@@ -643,12 +688,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                                             kc.h, kc.qu * UNIT_ROWS + qi * BM, kc.b);
                     }
                     if (!(ok = waiter.wait(bar(B_K_EMPTY + kr.s), kr.ph ^ 1, ROLE_TMA))) break;
-                    mbar_arrive_expect_tx(bar(B_K_FULL + kr.s), TILE_BYTES);
-                    armed_k |= 1u << kr.s;
-                    par_k = (par_k & ~(1u << kr.s)) | (kr.ph << kr.s);
-                    for (int bx = 0; bx < 2; ++bx)
-                        tma_load_4d(sK + kr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + kr.s), bx * 64,
-                                    kc.h, kj * BN, kc.b);
+                    // test hook: CTA 0 leaves one K tile unloaded, so that the
+                    // next wait for it runs out
+                    if (!(p.withhold_k >= 0 && blockIdx.x == 0 && kt == static_cast<uint32_t>(p.withhold_k))) {
+                        mbar_arrive_expect_tx(bar(B_K_FULL + kr.s), TILE_BYTES);
+                        armed_k |= 1u << kr.s;
+                        par_k = (par_k & ~(1u << kr.s)) | (kr.ph << kr.s);
+                        for (int bx = 0; bx < 2; ++bx)
+                            tma_load_4d(sK + kr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + kr.s),
+                                        bx * 64, kc.h, kc.tile(kj) * BN, kc.b);
+                    }
                     kr.next();
                     ++kt;
                     if (++kj == kc.nt) {
@@ -665,7 +714,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 par_v = (par_v & ~(1u << vr.s)) | (vr.ph << vr.s);
                 for (int bx = 0; bx < 2; ++bx)
                     tma_load_4d(sV + vr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_v, bar(B_V_FULL + vr.s), bx * 64,
-                                vc.h, vj * BN, vc.b);
+                                vc.h, vc.tile(vj) * BN, vc.b);
                 vr.next();
                 ++vt;
                 if (++vj == vc.nt) {
@@ -678,7 +727,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 // Abort: let every copy this warp started land before the CTA
                 // (and its shared memory) goes away.
                 volatile int never = 0;
-                Waiter tail{&never, 20000000ull};
+                Waiter tail{&never, 20000000ull, nullptr, false};
                 if (armed_q) tail.wait(bar(B_Q_FULL), par_q, ROLE_TMA);
                 for (int s = 0; s < p.kstages; ++s)
                     if ((armed_k >> s) & 1u) tail.wait(bar(B_K_FULL + s), (par_k >> s) & 1u, ROLE_TMA);
@@ -749,7 +798,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 // Abort: wait for the MMAs already issued before TMEM is freed.
                 mma_commit(bar(B_DRAIN));
                 volatile int never = 0;
-                Waiter tail{&never, 20000000ull};
+                Waiter tail{&never, 20000000ull, nullptr, false};
                 tail.wait(bar(B_DRAIN), 0, ROLE_MMA);
             }
         }
@@ -767,6 +816,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         const uint32_t tS = tmem_base + lane_off + TM_S + 128 * qi;
         const uint32_t tO = tmem_base + lane_off + TM_O + 128 * qi;
         const float sl2 = p.scale_log2;
+        // turns: warpgroup 0 takes the first; its n-th wait is for parity
+        // (n & 1) ^ 1 of its barrier (immediate for n = 0), warpgroup 1's for
+        // parity n & 1 (completed by warpgroup 0's n-th hand-off)
+        const uint32_t turn_flip = qi == 0 ? 1u : 0u;
         uint32_t sp = 0, lu = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
@@ -782,7 +835,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 tmem_wait_ld();
 #pragma unroll
                 for (int ch = 0; ch < BN / 32; ++ch) reg_fence32(sr + 32 * ch);
-                if (j == c.nt - 1) {
+                if (c.tile(j) == c.nt - 1) {
                     // key mask: columns at or past N + valid in the last tile
 #pragma unroll
                     for (int e = 0; e < BN; ++e)
@@ -807,6 +860,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     alpha = ex2_approx(m - m_new);
                 }
                 const float nm = -m_new;
+                // the exponentials: this warpgroup's turn on the MUFU units
+                if (!(ok = waiter.wait_warp(bar(B_TURN + qi), (sp & 1) ^ turn_flip, ROLE_SOFTMAX))) break;
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
                 for (int e = 0; e < BN; e += 4) {
@@ -822,6 +877,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     sr[e / 2] = pack_bf16x2(x0, x1);
                     sr[e / 2 + 1] = pack_bf16x2(x2, x3);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_TURN + (qi ^ 1)));
                 tmem_st32(tS, sr);
                 tmem_st32(tS + 32, sr + 32);
                 l = l * alpha + ((a0 + a1) + (a2 + a3));
@@ -849,18 +906,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 if (lane == 0) mbar_arrive(bar(B_P_READY + qi));
             }
             if (!ok) break;
-            // epilogue: out = O / l as bf16, one 256-byte row per thread
+            // epilogue: out = O / l, one row per thread
             if (!(ok = waiter.wait_warp(bar(B_O_DONE + qi), lu & 1, ROLE_SOFTMAX))) break;
             tc_fence_after();
             const float inv_l = 1.f / l;
             const int srow = c.qu * UNIT_ROWS + qi * BM + row;
             const bool store = srow < p.S;
+            const size_t orow = (static_cast<size_t>(c.b) * p.S + (store ? srow : 0)) * p.H + c.h;
             if constexpr (BLOCK) {
-                if (p.lse != nullptr && store)
-                    p.lse[(static_cast<size_t>(c.b) * p.S + srow) * p.H + c.h] = (m + log2f(l)) * 0.6931471805599453f;
+                if (p.lse != nullptr && store) p.lse[orow] = (m + log2f(l)) * 0.6931471805599453f;
+                if (p.out_f32) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D);
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld32(tO + 32 * ch, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
+                        if (store) {
+#pragma unroll
+                            for (int v4 = 0; v4 < 8; ++v4)
+                                dst[ch * 8 + v4] = make_float4(
+                                    __uint_as_float(r[4 * v4]) * inv_l, __uint_as_float(r[4 * v4 + 1]) * inv_l,
+                                    __uint_as_float(r[4 * v4 + 2]) * inv_l, __uint_as_float(r[4 * v4 + 3]) * inv_l);
+                        }
+                    }
+                    tc_fence_before();
+                    continue;
+                }
             }
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.out + ((static_cast<size_t>(c.b) * p.S + (store ? srow : 0)) * p.H + c.h) * D);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t r[32];
@@ -958,9 +1033,11 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
 // softmax over the union of the keys: with m = max(lse_acc, lse_part),
 // w = exp(lse - m), o_acc = (w_acc o_acc + w_part o_part) / (w_acc + w_part)
 // and lse_acc = m + log(w_acc + w_part). A block with lse = -inf adds nothing.
-// One warp per 128-channel row; optionally writes the merged row as bf16.
+// o_part is fp32 (PART_F32) or bf16. One warp per 128-channel row;
+// optionally writes the merged row as bf16.
+template <bool PART_F32>
 __global__ void __launch_bounds__(256) hv_merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
-                                                       const uint2* __restrict__ o_part,
+                                                       const void* __restrict__ o_part,
                                                        const float* __restrict__ lse_part, uint2* __restrict__ out,
                                                        long long rows) {
     const int lane = threadIdx.x & 31;
@@ -975,9 +1052,15 @@ __global__ void __launch_bounds__(256) hv_merge_kernel(float* __restrict__ o_acc
         if (m != -INFINITY) {
             const float wa = expf(la - m), wb = expf(lb - m);
             const float tot = wa + wb;
-            const uint2 pb = o_part[r * 32 + lane];
-            const float b0 = __uint_as_float(pb.x << 16), b1 = __uint_as_float(pb.x & 0xFFFF0000u);
-            const float b2 = __uint_as_float(pb.y << 16), b3 = __uint_as_float(pb.y & 0xFFFF0000u);
+            float b0, b1, b2, b3;
+            if constexpr (PART_F32) {
+                const float4 pb = reinterpret_cast<const float4*>(o_part)[r * 32 + lane];
+                b0 = pb.x; b1 = pb.y; b2 = pb.z; b3 = pb.w;
+            } else {
+                const uint2 pb = reinterpret_cast<const uint2*>(o_part)[r * 32 + lane];
+                b0 = __uint_as_float(pb.x << 16); b1 = __uint_as_float(pb.x & 0xFFFF0000u);
+                b2 = __uint_as_float(pb.y << 16); b3 = __uint_as_float(pb.y & 0xFFFF0000u);
+            }
             const float inv = 1.f / tot;
             a.x = (a.x * wa + b0 * wb) * inv;
             a.y = (a.y * wa + b1 * wb) * inv;
@@ -991,7 +1074,7 @@ __global__ void __launch_bounds__(256) hv_merge_kernel(float* __restrict__ o_acc
     }
 }
 
-__global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns) {
+__global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns, unsigned int* status) {
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
@@ -1000,7 +1083,7 @@ __global__ void hv_selftest_timeout_kernel(unsigned long long timeout_ns) {
         fence_mbar_init();
     }
     __syncthreads();
-    const Waiter w{&abort_flag, timeout_ns};
+    const Waiter w{&abort_flag, timeout_ns, status};
     w.wait_warp(smem_addr(&mbar), 0, ROLE_SELFTEST);
     __syncthreads();
 }
@@ -1021,16 +1104,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [B, S, H, 128] bf16 as a 4-D tensor (channel, head, token, batch); a box is
-// 64 channels x 1 head x 128 tokens, landing as 128 rows of 128 bytes with the
-// 128-byte swizzle the MMA descriptors expect. Rows past S read as zero.
-static bool make_qkv_map(CUtensorMap* map, const void* ptr, int B, int S, int H) {
+// 64 channels x 1 head x box_rows tokens, landing as box_rows rows of 128
+// bytes with the 128-byte swizzle the MMA descriptors expect. Rows past S
+// read as zero.
+static bool make_qkv_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
                                 static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
                                    static_cast<cuuint64_t>(S) * H * D * 2};
-    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(BM), 1};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1087,10 +1171,53 @@ static bool ranges_overlap(const void* a, size_t a_bytes, const void* b, size_t 
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 
+// Host-visible status words, one 64-byte line per device ordinal, in a static
+// page of host memory that is page-locked and mapped into the device's
+// address space at first use (registration, not an allocation). A kernel
+// wait that runs out stores its code there, so that every later call sees
+// it without synchronising; hv_attn_last_device_error clears it.
+struct alignas(4096) StatusPage {
+    unsigned int word[64 * 16];
+};
+static StatusPage g_status_page;
+static std::mutex g_status_mu;
+
+static unsigned int* status_host(int dev) { return &g_status_page.word[(dev & 63) * 16]; }
+
+// Device address of this device's status word (the current device must be
+// `dev`), or nullptr if the page cannot be mapped (then only the device error
+// word records a timeout).
+static unsigned int* status_word_dev(int dev) {
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    void* dptr = nullptr;
+    if (cudaHostGetDevicePointer(&dptr, status_host(dev), 0) == cudaSuccess) return static_cast<unsigned int*>(dptr);
+    (void)cudaGetLastError();   // not registered (yet, or no longer): not an error of the call
+    if (cudaHostRegister(&g_status_page, sizeof(g_status_page), cudaHostRegisterMapped | cudaHostRegisterPortable) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    if (cudaHostGetDevicePointer(&dptr, status_host(dev), 0) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    return static_cast<unsigned int*>(dptr);
+}
+
+static bool status_timed_out(int dev) { return *static_cast<volatile unsigned int*>(status_host(dev)) != 0u; }
+
 struct Call {
-    int S = 0, N = 0, sms = 0;
+    int S = 0, N = 0, sms = 0, dev = 0;
     long long units = 0;
     size_t bytes = 0;   // bytes of one [B, S, heads, 128] bf16 tensor
+};
+
+// Options of one launch of the attention kernel beyond the call's arguments.
+struct LaunchOpts {
+    unsigned long long timeout_ns = kWaitTimeoutNs;
+    int withhold_k = -1;   // test hook of hv_attn_selftest_abort
+    int h_total = 0;       // heads of the whole call (0: this launch's), for a launch over a head group
+    int h_offset = 0;      // first head of the group within the call
 };
 
 // Checks of the QK RMSNorm arguments: gamma (device, fp32 [4][128], 16-byte
@@ -1132,9 +1259,11 @@ static int validate(const void* q, const void* k, const void* v, const void* out
     if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
     DeviceInfo& di = device_info(dev);
     if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    if (status_timed_out(dev)) return HV_ERR_DEVICE_TIMEOUT;
     call.S = static_cast<int>(s_len);
     call.N = static_cast<int>(n_video);
     call.sms = di.sms;
+    call.dev = dev;
     call.units = units;
     call.bytes = bytes;
     return HV_OK;
@@ -1163,23 +1292,24 @@ struct Blocks {
     int Sk, q_vid, q_pos0, k_vid, k_pos0;
     const int* kv_len;   // host, B entries, each in [1, Sk]
     float* lse;          // device or nullptr
+    int out_f32;         // 1: out rows are fp32
 };
 
 static int launch_attention(const Call& call, const void* q, const void* k, const void* v, void* out, int B,
                             int heads, int T, int Hp, int Wp, int text_len, const int* text_valid, float rope_theta,
                             float scale, bool k_rotated, const float* qk_gamma, float qk_eps,
-                            cudaStream_t stream, const Blocks* blk = nullptr) {
+                            cudaStream_t stream, const Blocks* blk = nullptr, const LaunchOpts& opts = LaunchOpts()) {
     (void)text_len;
     Params* prm = new Params;   // ~2.5 KB; heap to keep the host stack small
     std::memset(prm, 0, sizeof(Params));
     const int S = call.S;
     const int Sk = blk ? blk->Sk : S;
-    if (!make_qkv_map(&prm->tm_q, q, B, S, heads) || !make_qkv_map(&prm->tm_k, k, B, Sk, heads) ||
-        !make_qkv_map(&prm->tm_v, v, B, Sk, heads)) {
+    if (!make_qkv_map(&prm->tm_q, q, B, S, heads, BM) || !make_qkv_map(&prm->tm_k, k, B, Sk, heads, BN) ||
+        !make_qkv_map(&prm->tm_v, v, B, Sk, heads, BN)) {
         delete prm;
         return HV_ERR_LAUNCH;
     }
-    prm->out = static_cast<__nv_bfloat16*>(out);
+    prm->out = out;
     prm->B = B;
     prm->H = heads;
     prm->S = S;
@@ -1199,7 +1329,12 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->units = static_cast<int>(call.units);
     prm->theta_log2 = static_cast<float>(std::log2(static_cast<double>(rope_theta)));
     prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    prm->timeout_ns = kWaitTimeoutNs;
+    prm->timeout_ns = opts.timeout_ns;
+    prm->status = status_word_dev(call.dev);
+    prm->withhold_k = opts.withhold_k;
+    prm->h_total = opts.h_total > 0 ? opts.h_total : heads;
+    prm->h_offset = opts.h_offset;
+    prm->round_width = call.sms;
     prm->Sk = Sk;
     if (blk) {
         prm->q_vid = blk->q_vid;
@@ -1207,18 +1342,21 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
         prm->k_vid = blk->k_vid;
         prm->k_pos0 = blk->k_pos0;
         prm->lse = blk->lse;
+        prm->out_f32 = blk->out_f32;
         for (int b = 0; b < B; ++b) prm->kv_len[b] = blk->kv_len[b];
     } else {
         prm->q_vid = prm->k_vid = call.N;
         for (int b = 0; b < B; ++b) prm->kv_len[b] = call.N + text_valid[b];
     }
+    // persistent grid: one CTA per SM, at most one per work unit
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
     if (blk)
         hv_attn_fwd_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     else
         hv_attn_fwd_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    cudaError_t err = cudaSuccess;
     delete prm;
-    const cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) err = cudaGetLastError();
     return err == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
@@ -1439,8 +1577,12 @@ int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_h
         good = good && cudaStreamWaitEvent(cs, hp->h2d_done[slot], 0) == cudaSuccess &&
                cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
         if (good) {
+            LaunchOpts opts;
+            opts.h_total = heads;
+            opts.h_offset = g * hg;
             st = launch_attention(call, slot_buf(slot, 0), slot_buf(slot, 1), slot_buf(slot, 2), slot_buf(slot, 3), B,
-                                  hg, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false, nullptr, 0.f, cs);
+                                  hg, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false, nullptr, 0.f, cs,
+                                  nullptr, opts);
             if (st != HV_OK) return st;
         }
         good = good && cudaEventRecord(hp->comp_done[slot], cs) == cudaSuccess;
@@ -1457,13 +1599,14 @@ int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_h
 
 int hv_attn_forward_block(const void* q, const void* k, const void* v, void* out, float* lse, int B, int heads,
                           int T, int Hp, int Wp, int Sq, int q_video, int q_pos0, int Sk, int k_video, int k_pos0,
-                          const int* kv_len, float rope_theta, float scale, void* cuda_stream) {
+                          const int* kv_len, float rope_theta, float scale, int out_fp32, void* cuda_stream) {
     using namespace hv;
     if (!q || !k || !v || !out || !kv_len) return HV_ERR_NULL_POINTER;
     const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
     if ((mis & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return HV_ERR_MISALIGNED;
-    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH || Sq < 1 || Sk < 1)
+    if (B < 1 || heads < 1 || T < 1 || Hp < 1 || Wp < 1 || B > HV_MAX_BATCH || Sq < 1 || Sk < 1 ||
+        (out_fp32 != 0 && out_fp32 != 1))
         return HV_ERR_BAD_SHAPE;
     const long long n_video = static_cast<long long>(T) * Hp * Wp;
     if (q_video < 0 || q_video > Sq || k_video < 0 || k_video > Sk || q_pos0 < 0 || k_pos0 < 0 ||
@@ -1478,45 +1621,54 @@ int hv_attn_forward_block(const void* q, const void* k, const void* v, void* out
         n_video >= (1ll << 31))
         return HV_ERR_TOO_LARGE;
     const size_t qb = static_cast<size_t>(B) * Sq * heads * D * 2, kb = static_cast<size_t>(B) * Sk * heads * D * 2;
+    const size_t ob = out_fp32 ? 2 * qb : qb;
     const size_t lb = static_cast<size_t>(B) * Sq * heads * 4;
-    if (ranges_overlap(out, qb, q, qb) || ranges_overlap(out, qb, k, kb) || ranges_overlap(out, qb, v, kb))
+    if (ranges_overlap(out, ob, q, qb) || ranges_overlap(out, ob, k, kb) || ranges_overlap(out, ob, v, kb))
         return HV_ERR_ALIAS;
-    if (lse && (ranges_overlap(lse, lb, out, qb) || ranges_overlap(lse, lb, q, qb) || ranges_overlap(lse, lb, k, kb) ||
+    if (lse && (ranges_overlap(lse, lb, out, ob) || ranges_overlap(lse, lb, q, qb) || ranges_overlap(lse, lb, k, kb) ||
                 ranges_overlap(lse, lb, v, kb)))
         return HV_ERR_ALIAS;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
     DeviceInfo& di = device_info(dev);
     if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    if (status_timed_out(dev)) return HV_ERR_DEVICE_TIMEOUT;
     Call call;
     call.S = Sq;
     call.N = static_cast<int>(n_video);
     call.sms = di.sms;
+    call.dev = dev;
     call.units = units;
     call.bytes = qb;
-    const Blocks blk{Sk, q_video, q_pos0, k_video, k_pos0, kv_len, lse};
+    const Blocks blk{Sk, q_video, q_pos0, k_video, k_pos0, kv_len, lse, out_fp32};
     return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, 0, nullptr, rope_theta, scale, false, nullptr,
                             0.f, static_cast<cudaStream_t>(cuda_stream), &blk);
 }
 
-int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* out, long long rows,
-                  void* cuda_stream) {
+int hv_attn_merge(float* o_acc, float* lse_acc, const void* o_part, int o_part_fp32, const float* lse_part, void* out,
+                  long long rows, void* cuda_stream) {
     using namespace hv;
     if (!o_acc || !lse_acc || !o_part || !lse_part) return HV_ERR_NULL_POINTER;
-    if ((reinterpret_cast<uintptr_t>(o_acc) & 15u) || (reinterpret_cast<uintptr_t>(o_part) & 7u) ||
+    if ((reinterpret_cast<uintptr_t>(o_acc) & 15u) || (reinterpret_cast<uintptr_t>(o_part) & (o_part_fp32 ? 15u : 7u)) ||
         (reinterpret_cast<uintptr_t>(out) & 7u) || (reinterpret_cast<uintptr_t>(lse_acc) & 3u) ||
         (reinterpret_cast<uintptr_t>(lse_part) & 3u))
         return HV_ERR_MISALIGNED;
-    if (rows < 0) return HV_ERR_BAD_SHAPE;
+    if (rows < 0 || (o_part_fp32 != 0 && o_part_fp32 != 1)) return HV_ERR_BAD_SHAPE;
     if (rows == 0) return HV_OK;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HV_ERR_LAUNCH;
     DeviceInfo& di = device_info(dev);
     if (di.ok != 1) return HV_ERR_NO_DEVICE;
+    if (status_timed_out(dev)) return HV_ERR_DEVICE_TIMEOUT;
     const long long blocks = (rows + 7) / 8;
     const int grid = static_cast<int>(blocks < 16ll * di.sms ? blocks : 16ll * di.sms);
-    hv_merge_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-        o_acc, lse_acc, static_cast<const uint2*>(o_part), lse_part, static_cast<uint2*>(out), rows);
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (o_part_fp32)
+        hv_merge_kernel<true><<<grid, 256, 0, stream>>>(o_acc, lse_acc, o_part, lse_part, static_cast<uint2*>(out),
+                                                        rows);
+    else
+        hv_merge_kernel<false><<<grid, 256, 0, stream>>>(o_acc, lse_acc, o_part, lse_part, static_cast<uint2*>(out),
+                                                         rows);
     return cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
@@ -1525,15 +1677,39 @@ int hv_attn_last_device_error(void) {
     unsigned int word = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&word, hv::g_dev_error, sizeof(word)) != cudaSuccess) return -1;
     if (cudaMemcpyToSymbol(hv::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    *static_cast<volatile unsigned int*>(hv::status_host(dev)) = 0u;
     return static_cast<int>(word);
 }
 
 int hv_attn_selftest_timeout(int timeout_us) {
     if (timeout_us < 1 || timeout_us > 1000000) return -1;
-    if (hv_attn_last_device_error() < 0) return -1;   // clears the word first
-    hv::hv_selftest_timeout_kernel<<<1, 32>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+    if (hv_attn_last_device_error() < 0) return -1;   // clears the words first
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    hv::hv_selftest_timeout_kernel<<<1, 32>>>(static_cast<unsigned long long>(timeout_us) * 1000ull,
+                                              hv::status_word_dev(dev));
     if (cudaGetLastError() != cudaSuccess) return -1;
     return hv_attn_last_device_error();
+}
+
+int hv_attn_selftest_abort(const void* q, const void* k, const void* v, void* out, int B, int heads, int T, int Hp,
+                           int Wp, int text_len, const int* text_valid, int withhold_k, int timeout_us,
+                           void* cuda_stream) {
+    using namespace hv;
+    if (withhold_k < 0 || timeout_us < 1000 || timeout_us > 1000000) return HV_ERR_BAD_SCALAR;
+    Call call;
+    const int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, 256.f, 0.08838834764831843f, call);
+    if (st != HV_OK) return st;
+    LaunchOpts opts;
+    opts.timeout_ns = static_cast<unsigned long long>(timeout_us) * 1000ull;
+    opts.withhold_k = withhold_k;
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const int ls = launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, 256.f,
+                                    0.08838834764831843f, false, nullptr, 0.f, stream, nullptr, opts);
+    if (ls != HV_OK) return ls;
+    return cudaStreamSynchronize(stream) == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
 }
 
 }  // extern "C"

@@ -18,6 +18,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// store visible to the host (mapped pinned memory)
+__device__ __forceinline__ void st_sys_u32(unsigned int* p, uint32_t v) {
+    asm volatile("st.volatile.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    asm volatile("fence.sc.sys;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -29,7 +29,8 @@ EXPORTED = ("hv_attn_forward", "hv_attn_forward_ws", "hv_attn_forward_noalloc", 
             "hv_attn_forward_qknorm_ws", "hv_attn_forward_host", "hv_attn_host_workspace_bytes",
             "hv_attn_workspace_bytes", "hv_attn_forward_block", "hv_attn_merge",
             "hv_video_tokens",
-            "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_status_string")
+            "hv_attn_last_device_error", "hv_attn_selftest_timeout", "hv_attn_selftest_abort",
+            "hv_attn_status_string")
 
 
 class HVError(RuntimeError):
@@ -71,9 +72,13 @@ def lib() -> ctypes.CDLL:
         L.hv_attn_host_workspace_bytes.argtypes = [ctypes.c_int] * 7
         L.hv_attn_forward_block.restype = ctypes.c_int
         L.hv_attn_forward_block.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 11 + [
-            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
+            ctypes.POINTER(ctypes.c_int), ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
         L.hv_attn_merge.restype = ctypes.c_int
-        L.hv_attn_merge.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_longlong, ctypes.c_void_p]
+        L.hv_attn_merge.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] + [ctypes.c_void_p] * 2 + [
+            ctypes.c_longlong, ctypes.c_void_p]
+        L.hv_attn_selftest_abort.restype = ctypes.c_int
+        L.hv_attn_selftest_abort.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+            ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
         L.hv_attn_workspace_bytes.restype = ctypes.c_longlong
         L.hv_attn_workspace_bytes.argtypes = [ctypes.c_int] * 6
         L.hv_video_tokens.restype = ctypes.c_longlong
@@ -104,6 +109,25 @@ def last_device_error() -> int:
 
 def selftest_timeout(timeout_us: int = 20000) -> int:
     return int(lib().hv_attn_selftest_timeout(int(timeout_us)))
+
+
+def selftest_abort(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, text_valid,
+                   withhold_k: int = 1, timeout_us: int = 20000, out: torch.Tensor | None = None) -> int:
+    """``hv_attn_selftest_abort``: the attention kernel with one K load withheld and short
+    wait limits; returns the call's status (the timeout shows in the error words)."""
+    _check(q, "q")
+    _check(k, "k", q.shape)
+    _check(v, "v", q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    b_sz, _, heads, _ = q.shape
+    t_lat, hp, wp = (int(x) for x in grid)
+    valid = (ctypes.c_int * b_sz)(*[int(x) for x in text_valid])
+    stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        return int(lib().hv_attn_selftest_abort(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b_sz,
+                                                heads, t_lat, hp, wp, int(text_len), valid, int(withhold_k),
+                                                int(timeout_us), ctypes.c_void_p(stream.cuda_stream)))
 
 
 def _check(t: torch.Tensor, name: str, shape=None):
@@ -251,9 +275,10 @@ def attn_forward_qknorm(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid,
 def attn_forward_block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, q_video: int, q_pos0: int,
                        k_video: int, k_pos0: int, kv_len, rope_theta: float = 256.0, scale: float | None = None,
                        out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-                       stream: torch.cuda.Stream | None = None):
+                       out_dtype: torch.dtype = torch.float32, stream: torch.cuda.Stream | None = None):
     """One ring-attention step (``hv_attn_forward_block``): q [B, Sq, H, 128]
-    against k, v [B, Sk, H, 128]; returns (out bf16 [B, Sq, H, 128], lse fp32
+    against k, v [B, Sk, H, 128]; returns (out [B, Sq, H, 128] of ``out_dtype``:
+    fp32 (default, the partial result kept exact for merging) or bf16, lse fp32
     [B, Sq, H])."""
     _check(q, "q")
     _check(k, "k")
@@ -261,8 +286,10 @@ def attn_forward_block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, 
     if k.shape[0] != q.shape[0] or k.shape[2] != q.shape[2]:
         raise ValueError("q and k/v must agree in batch and heads")
     if out is None:
-        out = torch.empty_like(q)
-    _check(out, "out", q.shape)
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or not out.is_cuda or not out.is_contiguous() \
+            or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be a contiguous fp32 or bf16 CUDA tensor shaped like q")
     b_sz, sq, heads, _ = q.shape
     sk = k.shape[1]
     if lse is None:
@@ -281,6 +308,7 @@ def attn_forward_block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, 
         st = lib().hv_attn_forward_block(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                          b_sz, heads, t_lat, hp, wp, sq, int(q_video), int(q_pos0), sk,
                                          int(k_video), int(k_pos0), kvl, float(rope_theta), float(scale),
+                                         1 if out.dtype == torch.float32 else 0,
                                          ctypes.c_void_p(stream.cuda_stream))
     if st != HV_OK:
         raise HVError(st, "hv_attn_forward_block")
@@ -289,11 +317,12 @@ def attn_forward_block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, 
 
 def attn_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, lse_part: torch.Tensor,
                out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> None:
-    """``hv_attn_merge``: fold (o_part bf16, lse_part fp32) into (o_acc fp32, lse_acc fp32) in place;
-    optionally also write the merged rows to ``out`` (bf16)."""
+    """``hv_attn_merge``: fold (o_part fp32 or bf16, lse_part fp32) into (o_acc fp32, lse_acc fp32) in
+    place; optionally also write the merged rows to ``out`` (bf16)."""
     rows = lse_acc.numel()
+    part_dt = o_part.dtype if o_part.dtype in (torch.float32, torch.bfloat16) else torch.float32
     for name, t, dt in (("o_acc", o_acc, torch.float32), ("lse_acc", lse_acc, torch.float32),
-                        ("o_part", o_part, torch.bfloat16), ("lse_part", lse_part, torch.float32)):
+                        ("o_part", o_part, part_dt), ("lse_part", lse_part, torch.float32)):
         if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
     if o_acc.numel() != rows * 128 or o_part.numel() != rows * 128 or lse_part.numel() != rows:
@@ -303,7 +332,8 @@ def attn_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor,
     if stream is None:
         stream = torch.cuda.current_stream(o_acc.device)
     with torch.cuda.device(o_acc.device):
-        st = lib().hv_attn_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+        st = lib().hv_attn_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(),
+                                 1 if o_part.dtype == torch.float32 else 0, lse_part.data_ptr(),
                                  None if out is None else out.data_ptr(), rows, ctypes.c_void_p(stream.cuda_stream))
     if st != HV_OK:
         raise HVError(st, "hv_attn_merge")

@@ -12,9 +12,10 @@ Layout (one process per GPU, ``torch.distributed``):
   sequence (``ring_chunks``); rank r holds run r of Q, K and V, and the whole
   text segment (replicated);
 * step s: rank r attends its queries [run r ; text] to the K/V run of rank
-  r - s (``hv_attn_forward_block``, RoPE at the run's global token indices)
-  while it passes that run on to rank r + 1 and receives the next one;
-  ``hv_attn_merge`` folds each block into an fp32 accumulator;
+  r - s (``hv_attn_forward_block``, RoPE at the run's global token indices,
+  the block's result kept in fp32) while it passes that run on to rank r + 1
+  and receives the next one; ``hv_attn_merge`` folds each block into an fp32
+  accumulator, so no step of the ring rounds to bf16 before the last;
 * a last block attends to the text keys (padding masked per sample) and
   writes the bf16 output.
 

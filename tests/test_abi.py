@@ -141,23 +141,31 @@ def test_block_and_merge_entry_points_validate_arguments(lib):
     f = lib.hv_attn_forward_block
     q, k, v, o, lse = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
     grid = (2, 4, 4)                                   # 32 video tokens
-    ok = (1, 2, *grid, 40, 20, 0, 16, 16, 8, kv, 256.0, 0.088, None)
+    ok = (1, 2, *grid, 40, 20, 0, 16, 16, 8, kv, 256.0, 0.088, 1, None)
     assert f(None, k, v, o, lse, *ok) == 1
     assert f(q, k, v, o, lse + 2, *ok) == 2                                       # lse misaligned
-    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 41, 0, 16, 16, 8, kv, 256.0, 0.088, None) == 3   # q_video > Sq
-    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 13, 16, 16, 8, kv, 256.0, 0.088, None) == 3  # past the grid
-    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 17, kv, 256.0, 0.088, None) == 3  # k past the grid
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 41, 0, 16, 16, 8, kv, 256.0, 0.088, 1, None) == 3   # q_video > Sq
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 13, 16, 16, 8, kv, 256.0, 0.088, 1, None) == 3  # past the grid
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 17, kv, 256.0, 0.088, 1, None) == 3  # k past the grid
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, kv, 256.0, 0.088, 2, None) == 3   # out_fp32 not 0/1
     bad = (ctypes.c_int * 1)(17)
-    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, bad, 256.0, 0.088, None) == 4  # kv_len > Sk
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, bad, 256.0, 0.088, 1, None) == 4  # kv_len > Sk
     zero = (ctypes.c_int * 1)(0)
-    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, zero, 256.0, 0.088, None) == 4
+    assert f(q, k, v, o, lse, 1, 2, *grid, 40, 20, 0, 16, 16, 8, zero, 256.0, 0.088, 1, None) == 4
     assert f(q, k, v, q + 64, lse, *ok) == 6                                      # out over q
     assert f(q, k, v, o, o + 16, *ok) == 6                                        # lse over out
+    # an fp32 out is twice as long as a bf16 one: 1 x 40 x 2 x 128 x 4 bytes = 40960
+    assert f(q, k, v, o, o + 30000, *ok) == 6                                     # lse inside the fp32 out
+    bf16 = ok[:-2] + (0, None)
+    assert f(q, k, v, o, o + 30000, *bf16) != 6                                   # past the bf16 out
     m = lib.hv_attn_merge
-    assert m(None, 0x10, 0x20, 0x30, None, 4, None) == 1
-    assert m(0x1008, 0x10, 0x20, 0x30, None, 4, None) == 2                        # o_acc not 16-byte aligned
-    assert m(0x1000, 0x10, 0x20, 0x30, None, -1, None) == 3
-    assert m(0x1000, 0x10, 0x20, 0x30, None, 0, None) == 0                        # nothing to merge
+    assert m(None, 0x10, 0x20, 1, 0x30, None, 4, None) == 1
+    assert m(0x1008, 0x10, 0x20, 1, 0x30, None, 4, None) == 2                     # o_acc not 16-byte aligned
+    assert m(0x1000, 0x10, 0x28, 1, 0x30, None, 4, None) == 2                     # fp32 o_part not 16-byte aligned
+    assert m(0x1000, 0x10, 0x28, 0, 0x30, None, 0, None) == 0                     # bf16 o_part: 8 bytes suffice
+    assert m(0x1000, 0x10, 0x20, 1, 0x30, None, -1, None) == 3
+    assert m(0x1000, 0x10, 0x20, 2, 0x30, None, 4, None) == 3                     # o_part_fp32 not 0/1
+    assert m(0x1000, 0x10, 0x20, 1, 0x30, None, 0, None) == 0                     # nothing to merge
 
 
 def test_valid_arguments_without_gpu_fail_cleanly(lib):
@@ -167,6 +175,10 @@ def test_valid_arguments_without_gpu_fail_cleanly(lib):
     st = _call(lib, q=1 << 32, k=2 << 32, v=3 << 32, out=4 << 32)
     assert st in (8, 9)
     valid = (ctypes.c_int * 1)(5)
+    st = lib.hv_attn_selftest_abort(1 << 32, 2 << 32, 3 << 32, 4 << 32, 1, 2, 2, 4, 4, 8, valid, 1, 20000, None)
+    assert st in (8, 9)
+    assert lib.hv_attn_selftest_abort(1 << 32, 2 << 32, 3 << 32, 4 << 32, 1, 2, 2, 4, 4, 8, valid, -1, 20000,
+                                      None) == 7
     st = lib.hv_attn_forward_qknorm(1 << 32, 2 << 32, 3 << 32, 4 << 32, 1, 2, 2, 4, 4, 8, valid, 256.0, 0.088,
                                     5 << 32, 1e-6, None)
     assert st in (8, 9)

@@ -212,6 +212,29 @@ def test_bounded_wait_times_out_cleanly():
     full_check(inp, (2, 4, 4), 8)
 
 
+def test_attention_kernel_abort_path():
+    """The attention kernel's own abort path (hv_attn_selftest_abort): with one K
+    tile load of CTA 0 withheld and 20 ms wait limits, the RoPE warps' wait for
+    those keys runs out; that CTA's roles stop, drain their copies and MMAs,
+    free TMEM and return, while the other CTAs finish. The timeout
+    is then visible without synchronising: the next call returns
+    HV_ERR_DEVICE_TIMEOUT without launching, until hv_attn_last_device_error
+    reads the word (timeout bit, RoPE role) and clears it. A normal call
+    afterwards matches the oracle."""
+    grid, text_len = (2, 8, 20), 64            # 384 rows: two work units per head
+    inp = _small(grid, text_len, [40], heads=4)
+    q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
+    assert H.last_device_error() == 0
+    assert H.selftest_abort(q, k, v, grid, text_len, [40], withhold_k=1, timeout_us=20000) == 0
+    with pytest.raises(H.HVError) as e:
+        H.attn_forward(q, k, v, grid, text_len, [40])
+    assert e.value.status == 10
+    word = H.last_device_error()
+    assert word & 1 and (word >> 8) & 0x4, hex(word)
+    assert H.last_device_error() == 0
+    full_check(inp, grid, text_len)
+
+
 # ------------------------------------------------ workspace (pre-rotated K) path
 
 def _run_both(inp, grid, text_len, theta=256.0):

@@ -77,9 +77,13 @@ def test_whole_sequence_block_is_the_plain_call():
     q, k, v = (_dev(inp[n]) for n in ("q", "k", "v"))
     ref = H.attn_forward(q, k, v, wl.grid, wl.text_len, inp["text_valid"])
     n = wl.n_video
-    o, _ = H.attn_forward_block(q, k, v, wl.grid, n, 0, n, 0, [n + int(x) for x in inp["text_valid"]])
+    kv = [n + int(x) for x in inp["text_valid"]]
+    o, _ = H.attn_forward_block(q, k, v, wl.grid, n, 0, n, 0, kv, out_dtype=torch.bfloat16)
+    o32, _ = H.attn_forward_block(q, k, v, wl.grid, n, 0, n, 0, kv)
     torch.cuda.synchronize()
     assert torch.equal(o, ref)
+    # the fp32 partial is the same result before its rounding to bf16
+    assert o32.dtype == torch.float32 and torch.equal(o32.to(torch.bfloat16), ref)
 
 
 def test_merge_kernel_matches_rule():
@@ -104,6 +108,14 @@ def test_merge_kernel_matches_rule():
     assert np.array_equal(np.isinf(got_l), np.isinf(ref_l))
     np.testing.assert_allclose(got_l[np.isfinite(ref_l)], ref_l[np.isfinite(ref_l)], rtol=1e-5, atol=1e-5)
     np.testing.assert_allclose(out.float().cpu().numpy(), got_o, rtol=2 ** -8, atol=1e-6)
+    # fp32 partials (what the ring passes): merged without a bf16 rounding of the part
+    part_f = rng.standard_normal((rows, 128)).astype(np.float32)
+    ao2, al2 = torch.from_numpy(acc_o).cuda(), torch.from_numpy(acc_l).cuda()
+    H.attn_merge(ao2, al2, torch.from_numpy(part_f).cuda(), torch.from_numpy(part_l).cuda())
+    torch.cuda.synchronize()
+    ref_o2, _ = O.merge_blocks([acc_o.astype(np.float64), part_f.astype(np.float64)],
+                               [acc_l.astype(np.float64), part_l.astype(np.float64)])
+    np.testing.assert_allclose(ao2.cpu().numpy().astype(np.float64), ref_o2, rtol=1e-5, atol=1e-5)
 
 
 def _free_port() -> int:
