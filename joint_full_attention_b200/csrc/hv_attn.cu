@@ -22,12 +22,6 @@
 // bf16 probabilities P_i overwrite the first 64 columns of S_i and feed the
 // PV MMA straight from TMEM.
 //
-// The two softmax warpgroups take turns for their exponentials (an mbarrier
-// hand-off per K tile): the MUFU unit of each SM sub-partition then serves one
-// warpgroup at a time at its full rate, which keeps each Q tile's chain
-// (softmax, then PV and the next QK on the tensor core) short while the other
-// tile's MMAs run.
-//
 // Every mbarrier wait is bounded by a %globaltimer budget; when one runs out
 // the CTA records the role in a device error word and in a host-visible status
 // word, tells the other roles to stop, waits (bounded) for its own copies and
@@ -111,8 +105,7 @@ constexpr int B_V_EMPTY = B_V_FULL + VSTAGES_MAX;
 constexpr int B_S_FULL = B_V_EMPTY + VSTAGES_MAX;
 constexpr int B_P_READY = B_S_FULL + QTILES;
 constexpr int B_O_DONE = B_P_READY + QTILES;
-constexpr int B_TURN = B_O_DONE + QTILES;    // softmax warpgroup i may start its exponentials
-constexpr int B_DRAIN = B_TURN + QTILES;
+constexpr int B_DRAIN = B_O_DONE + QTILES;
 constexpr int NUM_BARS = B_DRAIN + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
@@ -625,7 +618,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             mbar_init(bar(B_S_FULL + i), 1);
             mbar_init(bar(B_P_READY + i), 4);
             mbar_init(bar(B_O_DONE + i), 1);
-            mbar_init(bar(B_TURN + i), 4);
         }
         mbar_init(bar(B_DRAIN), 1);
         *abort_flag = 0;
@@ -816,10 +808,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         const uint32_t tS = tmem_base + lane_off + TM_S + 128 * qi;
         const uint32_t tO = tmem_base + lane_off + TM_O + 128 * qi;
         const float sl2 = p.scale_log2;
-        // turns: warpgroup 0 takes the first; its n-th wait is for parity
-        // (n & 1) ^ 1 of its barrier (immediate for n = 0), warpgroup 1's for
-        // parity n & 1 (completed by warpgroup 0's n-th hand-off)
-        const uint32_t turn_flip = qi == 0 ? 1u : 0u;
         uint32_t sp = 0, lu = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++lu) {
@@ -860,8 +848,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     alpha = ex2_approx(m - m_new);
                 }
                 const float nm = -m_new;
-                // the exponentials: this warpgroup's turn on the MUFU units
-                if (!(ok = waiter.wait_warp(bar(B_TURN + qi), (sp & 1) ^ turn_flip, ROLE_SOFTMAX))) break;
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
                 for (int e = 0; e < BN; e += 4) {
@@ -877,8 +863,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     sr[e / 2] = pack_bf16x2(x0, x1);
                     sr[e / 2 + 1] = pack_bf16x2(x2, x3);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_TURN + (qi ^ 1)));
                 tmem_st32(tS, sr);
                 tmem_st32(tS + 32, sr + 32);
                 l = l * alpha + ((a0 + a1) + (a2 + a3));
