@@ -562,26 +562,21 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
 }
 
 // S_i = Q_i K^T: 8 MMAs of K=16 channels; both operands K-major, 128B swizzle.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_tile, uint32_t k_tile) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-        const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
-        const uint64_t b = smem_desc_sw128(k_tile + off, 16, 1024);
-        mma_ss(d_tmem, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
-    }
+// q_desc, k_desc: shared-memory descriptors of the tiles' first 16 channels.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+    mma_ss_k128<BOX_BYTES / 16>(d_tmem, q_desc, k_desc, IDESC_QK, 0u);
 }
 
 // O_i (+)= P_i V: 8 MMAs of K=16 keys; P from TMEM (2 bf16 per column),
 // V MN-major (channels contiguous): LBO = distance between the two 64-channel
-// boxes, SBO = 8 key rows.
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_tile, bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint64_t b = smem_desc_sw128(v_tile + kk * 16 * 128, BOX_BYTES, 1024);
-        mma_ts(d_tmem, p_tmem + kk * 8, b, IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
-    }
+// boxes, SBO = 8 key rows. v_desc: descriptor of the tile's first 16 keys.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate) {
+    mma_ts_k128(d_tmem, p_tmem, v_desc, IDESC_PV, accumulate ? 1u : 0u);
 }
+
+// Descriptor of a K-major operand tile (Q or K) and of an MN-major V tile.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile) { return smem_desc_sw128(tile, 16, 1024); }
+__device__ __forceinline__ uint64_t v_desc_of(uint32_t tile) { return smem_desc_sw128(tile, BOX_BYTES, 1024); }
 
 // BLOCK: a ring-attention block (Q and K/V rows at their own global offsets,
 // log-sum-exp and optionally fp32 output); the standard call is compiled
@@ -736,6 +731,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             // K tiles are ready for the tensor core once the RoPE warps have
             // rotated them, or, when they arrive rotated, once TMA lands them.
             const int k_ready = p.k_rotated ? B_K_FULL : B_K_READY;
+            // operand descriptors, computed once: the MMAs only add offsets
+            // (a stage's tile lies TILE_BYTES / 16 address units after the previous one)
+            const uint64_t dq0 = kmajor_desc(sQ), dq1 = kmajor_desc(sQ + TILE_BYTES);
+            const uint64_t dk0 = kmajor_desc(sK), dv0 = v_desc_of(sV);
+            auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (TILE_BYTES / 16)); };
+            auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (TILE_BYTES / 16)); };
             Ring kr(p.kstages), vr(p.vstages);
             uint32_t lu = 0;
             uint32_t pr[QTILES] = {0, 0};
@@ -745,40 +746,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 if (!(ok = waiter.wait(bar(B_Q_READY), lu & 1, ROLE_MMA))) break;
                 if (!(ok = waiter.wait(bar(k_ready + kr.s), kr.ph, ROLE_MMA))) break;
                 tc_fence_after();
-                issue_qk(tmem_base + TM_S + 0, sQ, sK + kr.s * TILE_BYTES);
+                issue_qk(tmem_base + TM_S + 0, dq0, dk(kr.s));
                 mma_commit(bar(B_S_FULL + 0));
-                issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, sK + kr.s * TILE_BYTES);
+                issue_qk(tmem_base + TM_S + 128, dq1, dk(kr.s));
                 mma_commit(bar(B_S_FULL + 1));
                 mma_commit(bar(B_K_EMPTY + kr.s));
                 kr.next();
                 if (c.nt == 1) mma_commit(bar(B_Q_EMPTY));
                 for (int j = 0; j < c.nt; ++j) {
                     if (!(ok = waiter.wait(bar(B_V_FULL + vr.s), vr.ph, ROLE_MMA))) break;
-                    const uint32_t v_tile = sV + vr.s * TILE_BYTES;
+                    const uint64_t v_d = dv(vr.s);
                     // Q tile 0: PV for tile j, then QK for tile j+1
                     if (!(ok = waiter.wait(bar(B_P_READY + 0), pr[0] & 1, ROLE_MMA))) break;
                     ++pr[0];
                     tc_fence_after();
-                    issue_pv(tmem_base + TM_O + 0, tmem_base + TM_S + 0, v_tile, j > 0);
+                    issue_pv(tmem_base + TM_O + 0, tmem_base + TM_S + 0, v_d, j > 0);
                     if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 0));
                     const bool more = j + 1 < c.nt;
-                    const uint32_t k_tile = sK + kr.s * TILE_BYTES;
+                    const uint64_t k_d = dk(kr.s);
                     if (more) {
                         if (!(ok = waiter.wait(bar(k_ready + kr.s), kr.ph, ROLE_MMA))) break;
                         tc_fence_after();
-                        issue_qk(tmem_base + TM_S + 0, sQ, k_tile);
+                        issue_qk(tmem_base + TM_S + 0, dq0, k_d);
                         mma_commit(bar(B_S_FULL + 0));
                     }
                     // Q tile 1
                     if (!(ok = waiter.wait(bar(B_P_READY + 1), pr[1] & 1, ROLE_MMA))) break;
                     ++pr[1];
                     tc_fence_after();
-                    issue_pv(tmem_base + TM_O + 128, tmem_base + TM_S + 128, v_tile, j > 0);
+                    issue_pv(tmem_base + TM_O + 128, tmem_base + TM_S + 128, v_d, j > 0);
                     mma_commit(bar(B_V_EMPTY + vr.s));
                     vr.next();
                     if (j == c.nt - 1) mma_commit(bar(B_O_DONE + 1));
                     if (more) {
-                        issue_qk(tmem_base + TM_S + 128, sQ + TILE_BYTES, k_tile);
+                        issue_qk(tmem_base + TM_S + 128, dq1, k_d);
                         mma_commit(bar(B_S_FULL + 1));
                         mma_commit(bar(B_K_EMPTY + kr.s));
                         kr.next();
