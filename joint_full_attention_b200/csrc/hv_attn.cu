@@ -531,7 +531,8 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
     uint32_t lu = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
         const UnitCoord c = decode_unit(p, u);
-        if (!waiter.wait_warp(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
+        // every lane tests the barriers itself (a lane-0 wait and a broadcast cost more)
+        if (!waiter.wait(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
             if (p.qk_norm)
@@ -546,7 +547,7 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         bool ok = true;
         if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
         for (int j = 0; j < c.nt; ++j, kr.next()) {
-            if (!(ok = waiter.wait_warp(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
+            if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
             const int k0 = c.tile(j) * BN;
             if (p.qk_norm)
                 rope_norm_tile<BN>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, k0, k_vid,
@@ -816,7 +817,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             float m = -INFINITY;   // running max, scaled log2 units
             float l = 0.f;         // running sum of probabilities
             for (int j = 0; j < c.nt; ++j, ++sp) {
-                if (!(ok = waiter.wait_warp(bar(B_S_FULL + qi), sp & 1, ROLE_SOFTMAX))) break;
+                // every lane tests the barrier itself: no broadcast on the critical path
+                if (!(ok = waiter.wait(bar(B_S_FULL + qi), sp & 1, ROLE_SOFTMAX))) break;
                 tc_fence_after();
                 uint32_t sr[BN];
 #pragma unroll
