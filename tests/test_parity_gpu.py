@@ -8,6 +8,7 @@ on 4096 seeded (batch, head, row) samples for the two 129-frame workloads.
 
 from __future__ import annotations
 
+import ctypes
 import math
 
 import numpy as np
@@ -226,9 +227,29 @@ def test_attention_kernel_abort_path():
     q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
     assert H.last_device_error() == 0
     assert H.selftest_abort(q, k, v, grid, text_len, [40], withhold_k=1, timeout_us=20000) == 0
-    with pytest.raises(H.HVError) as e:
-        H.attn_forward(q, k, v, grid, text_len, [40])
-    assert e.value.status == 10
+    # every entry point that launches work refuses while the status word is set
+    gam = torch.ones((4, 128), dtype=torch.float32, device="cuda")
+    n = grid[0] * grid[1] * grid[2]
+    acc_o = torch.zeros((1, n + text_len, 4, 128), dtype=torch.float32, device="cuda")
+    acc_l = torch.full((1, n + text_len, 4), float("-inf"), dtype=torch.float32, device="cuda")
+    refused = [
+        lambda: H.attn_forward(q, k, v, grid, text_len, [40]),
+        lambda: H.attn_forward_ws(q, k, v, grid, text_len, [40]),
+        lambda: H.attn_forward_qknorm(q, k, v, grid, text_len, [40], gam),
+        lambda: H.attn_forward_qknorm(q, k, v, grid, text_len, [40], gam, use_workspace=True),
+        lambda: H.attn_forward_block(q, k, v, grid, n, 0, n, 0, [n + 40]),
+        lambda: H.attn_merge(acc_o, acc_l, acc_o.clone(), acc_l.clone()),
+    ]
+    for call in refused:
+        with pytest.raises(H.HVError) as e:
+            call()
+        assert e.value.status == 10
+    b_sz, _, heads, _ = q.shape
+    valid = (ctypes.c_int * 1)(40)
+    st = H.lib().hv_attn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), torch.empty_like(q).data_ptr(),
+                                         b_sz, heads, *grid, text_len, valid, 256.0, 1.0 / math.sqrt(128),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 10
     word = H.last_device_error()
     assert word & 1 and (word >> 8) & 0x4, hex(word)
     assert H.last_device_error() == 0
