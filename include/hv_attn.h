@@ -136,9 +136,20 @@ int hv_attn_forward_ws(const void* q, const void* k, const void* v, void* out,
  *            rows, in that order; shared by all heads. Must not overlap out.
  * qk_eps   : epsilon inside the root (finite, >= 0; the pages give no value,
  *            1e-6 is usual).
- * Other arguments, ownership, asynchrony and errors as hv_attn_forward;
+ * Other arguments, asynchrony and errors as hv_attn_forward;
  * HV_ERR_NULL_POINTER / HV_ERR_MISALIGNED / HV_ERR_BAD_SCALAR / HV_ERR_ALIAS
  * also cover qk_gamma and qk_eps.
+ *
+ * Two kernels: the first computes every key row's factor 1/rms once (reads
+ * K once), the attention kernel scales each K tile by them as it lands,
+ * instead of reducing every key row again for every 256-row query unit.
+ * Ownership: the caller owns all buffers. The row factors take
+ * 4 * B * heads * ceil(S/128) * 128 bytes of stream-ordered scratch
+ * (cudaMallocAsync on cuda_stream from the device's default memory pool,
+ * cudaFreeAsync on the same stream right after the attention kernel is
+ * enqueued); if the pool cannot provide it the call returns HV_ERR_LAUNCH
+ * before launching anything. Callers that must not allocate use
+ * hv_attn_forward_qknorm_ws with a workspace of their own.
  */
 int hv_attn_forward_qknorm(const void* q, const void* k, const void* v, void* out,
                            int B, int heads, int T, int Hp, int Wp,
@@ -152,7 +163,8 @@ int hv_attn_forward_qknorm(const void* q, const void* k, const void* v, void* ou
  * into `workspace` (text rows normalised), the attention kernel normalises
  * and rotates Q on load. Output bit-identical to hv_attn_forward_qknorm.
  * Arguments as hv_attn_forward_qknorm plus workspace / workspace_bytes as in
- * hv_attn_forward_ws (the workspace must not overlap qk_gamma either).
+ * hv_attn_forward_ws (the workspace must not overlap qk_gamma either). It
+ * allocates no device memory.
  */
 int hv_attn_forward_qknorm_ws(const void* q, const void* k, const void* v, void* out,
                               int B, int heads, int T, int Hp, int Wp,

@@ -74,11 +74,14 @@ constexpr int ROPE_THREADS = 192;
 constexpr int ROPE_WARPS = ROPE_THREADS / 32;
 constexpr int ROPE_GROUPS = ROPE_THREADS / 16;   // rows rb, rb + 12, rb + 24, ... per thread
 // per-thread registers after setmaxnreg: 2 x 128 x 176 + 128 x 64 + 128 x 96
-// = 65536 = 512 threads x 128 registers at launch
+// = 65536 = 512 threads x 128 registers at launch. With the QK RMSNorm
+// prologue the RoPE warps carry the normalisation too and take 80, the
+// control warpgroup 80.
 constexpr uint32_t REGS_SOFTMAX = 176;
-constexpr uint32_t REGS_ROPE = 64;
-constexpr uint32_t REGS_CONTROL = 96;
-static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL <= NUM_WARPS * 32 * 128,
+__host__ __device__ constexpr uint32_t regs_rope(bool qkn) { return qkn ? 80u : 64u; }
+__host__ __device__ constexpr uint32_t regs_control(bool qkn) { return qkn ? 80u : 96u; }
+__host__ __device__ constexpr uint32_t regs_split(bool qkn) { return 2 * 128 * REGS_SOFTMAX + 128 * regs_rope(qkn) + 128 * regs_control(qkn); }
+static_assert(regs_split(false) <= NUM_WARPS * 32 * 128 && regs_split(true) <= NUM_WARPS * 32 * 128,
               "register split exceeds the launch allocation");
 
 // shared memory map (offsets from a 1024-byte aligned base)
@@ -108,7 +111,10 @@ constexpr int B_O_DONE = B_P_READY + QTILES;
 constexpr int B_DRAIN = B_O_DONE + QTILES;
 constexpr int NUM_BARS = B_DRAIN + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_USED = OFF_MISC + 16;
+// 1/rms of the 128 rows of each K stage (QK RMSNorm with per-row statistics)
+constexpr int KR_BYTES = BN * 4;
+constexpr int OFF_KR = (OFF_MISC + 16 + 127) & ~127;
+constexpr int SMEM_USED = OFF_KR + KSTAGES_MAX * KR_BYTES;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-block limit");
 
@@ -132,9 +138,15 @@ struct __align__(64) Params {
     int B, H, S, N, T, Hp, Wp, HpWp;
     int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
     int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
-    int qk_norm;        // 1: RMSNorm the Q and K rows (gammas below) before rotating them
     float qk_eps;       // RMSNorm epsilon
     const float* qk_gamma;   // device, fp32 [4][128]: Q video, K video, Q text, K text
+    // Optional, with the QK RMSNorm: 1/rms of every K row, fp32 [B, H, k_rinv_ld]
+    // (k_rinv_ld a multiple of 128, entries past the rows 0), computed once
+    // per call by hv_k_rinv_kernel; the producer copies each K tile's 128
+    // values beside it and the RoPE warps scale by them instead of reducing
+    // every row again for every unit.
+    const float* k_rinv;
+    int k_rinv_ld;
     int kstages;        // K tiles in flight (slots 0 .. kstages-1 of the KV pool)
     int vstages;        // V tiles in flight (the next vstages slots)
     int n_qunits;       // ceil(S / 256)
@@ -331,28 +343,46 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) 
 // QK RMSNorm of one row ("HunyuanVideo 模型结构与数学原理" §5.4):
 // y = gamma * x / sqrt(mean_j x_j^2 + eps) over the 128 channels. The row's 16
 // chunks of 8 channels sit in the 16 lanes of one half-warp (lane & 15 =
-// chunk); every lane of the warp must call this together. The sum of squares
-// is taken in a fixed order (channel order, then a butterfly over the half-
-// warp), so every kernel that normalises a row this way gets the same bits.
-__device__ __forceinline__ void rms_norm_chunk(uint4 d, float4 g0, float4 g1, float eps, float (&y)[8]) {
+// chunk). The sum of squares is taken in a fixed order (channel order inside
+// a chunk, then a butterfly over the half-warp), so every kernel that
+// normalises a row this way gets the same bits.
+__device__ __forceinline__ void unpack_bf16x8(uint4 d, float (&x)[8]) {
     const uint32_t w[4] = {d.x, d.y, d.z, d.w};
-    float x[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         x[2 * q] = __uint_as_float(w[q] << 16);
         x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
     }
+}
+
+// 1/rms of the row: every lane of the warp must call this together.
+__device__ __forceinline__ float row_rms_inv(uint4 d, float eps) {
+    float x[8];
+    unpack_bf16x8(d, x);
     float ss = __fmul_rn(x[0], x[0]);
 #pragma unroll
     for (int c = 1; c < 8; ++c) ss = __fmaf_rn(x[c], x[c], ss);
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
-    const float r = rsqrtf(__fmaf_rn(ss, 1.f / D, eps));
-    const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-    for (int c = 0; c < 8; ++c) y[c] = __fmul_rn(__fmul_rn(x[c], r), g[c]);
+    return rsqrtf(__fmaf_rn(ss, 1.f / D, eps));
 }
 
+// y = (x * r) * gamma for the chunk's eight channels, two at a time.
+__device__ __forceinline__ void rms_scale_chunk(uint4 d, float r, uint4 g0, uint4 g1, float (&y)[8]) {
+    float x[8];
+    unpack_bf16x8(d, x);
+    const uint32_t g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+        float t0, t1;
+        fmul2(t0, t1, x[c], x[c + 1], r, r);
+        fmul2(y[c], y[c + 1], t0, t1, __uint_as_float(g[c]), __uint_as_float(g[c + 1]));
+    }
+}
+
+__device__ __forceinline__ void rms_norm_chunk(uint4 d, uint4 g0, uint4 g1, float eps, float (&y)[8]) {
+    rms_scale_chunk(d, row_rms_inv(d, eps), g0, g1, y);
+}
 
 __device__ __forceinline__ uint4 rotate_chunk(uint4 d, uint4 c, uint4 sn) {
     d.x = rotate_pair(d.x, __uint_as_float(c.x), __uint_as_float(sn.x));
@@ -450,13 +480,16 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 // tile of ROWS rows (rows rb, rb + 12, ...); text rows and rows past the
 // sequence are only normalised (rows past the sequence hold TMA's zero fill
 // and stay zero). gamma_v / gamma_t: shared-memory addresses of the video /
-// text gamma of this tensor (Q or K). Every lane of a warp runs the same
-// number of iterations (rb and rb + 1 share a warp, and as ROWS is even they
-// share a trip count), as the row sum is a half-warp shuffle.
+// text gamma of this tensor (Q or K). k_rinv: shared-memory address of the
+// tile's 128 row factors 1/rms when they were computed beforehand (K tiles
+// with per-row statistics), else 0 and each row's sum is reduced here, a
+// half-warp shuffle: then every lane of a warp runs the same number of
+// iterations (rb and rb + 1 share a warp, and as ROWS is even they share a
+// trip count).
 template <int ROWS>
 __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
-                                               int n0, int vid, int pos0, int rt, const RopeLane& L,
-                                               const Params& p) {
+                                               uint32_t k_rinv, int n0, int vid, int pos0, int rt,
+                                               const RopeLane& L, const Params& p) {
     static_assert(ROWS % 2 == 0, "half-warp row pairs");
     const int rb = rt >> 4;
     int n = n0 + rb;
@@ -470,14 +503,18 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
     const int stride = 2 * L.half_dim;
     const uint32_t gofs = 4u * static_cast<uint32_t>(L.ch0);
+    const uint4 gv0 = lds128(gamma_v + gofs), gv1 = lds128(gamma_v + gofs + 16);
 #pragma unroll 1
     for (int r = rb; r < ROWS; r += ROPE_GROUPS) {
         const bool video = n < vid;
         const int pos = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
         const uint32_t a = box_base + r * 128 + ((L.cin ^ (r & 7)) << 4);
         const uint4 d = lds128(a);
-        const uint32_t gb = (video ? gamma_v : gamma_t) + gofs;
-        const uint4 g0 = lds128(gb), g1 = lds128(gb + 16);
+        uint4 g0 = gv0, g1 = gv1;
+        if (!video) {
+            g0 = lds128(gamma_t + gofs);
+            g1 = lds128(gamma_t + gofs + 16);
+        }
         uint4 c = make_uint4(0u, 0u, 0u, 0u), sn = c;
         if (video && p.use_table) {
             const uint32_t t = tab + 4u * static_cast<uint32_t>(pos * stride);
@@ -485,11 +522,8 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
             sn = lds128(t + sin_off);
         }
         float y[8];
-        rms_norm_chunk(d, make_float4(__uint_as_float(g0.x), __uint_as_float(g0.y), __uint_as_float(g0.z),
-                                      __uint_as_float(g0.w)),
-                       make_float4(__uint_as_float(g1.x), __uint_as_float(g1.y), __uint_as_float(g1.z),
-                                   __uint_as_float(g1.w)),
-                       p.qk_eps, y);
+        const float rr = k_rinv ? lds_f32(k_rinv + 4u * static_cast<uint32_t>(r)) : row_rms_inv(d, p.qk_eps);
+        rms_scale_chunk(d, rr, g0, g1, y);
         uint32_t w[4];
         if (video) {
             if (p.use_table) {
@@ -519,9 +553,9 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
 
 // The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
 // each to the MMA warp.
-template <bool BLOCK>
+template <bool BLOCK, bool QKN>
 __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
-                                          uint32_t sK, uint32_t sTable, uint32_t sGamma) {
+                                          uint32_t sK, uint32_t sTable, uint32_t sGamma, uint32_t sKR) {
     const int q_vid = BLOCK ? p.q_vid : p.N, q_pos0 = BLOCK ? p.q_pos0 : 0;
     const int k_vid = BLOCK ? p.k_vid : p.N, k_pos0 = BLOCK ? p.k_pos0 : 0;
     const RopeLane L = make_rope_lane(rt, p);
@@ -535,9 +569,9 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         if (!waiter.wait(bar(B_Q_FULL), lu & 1, ROLE_ROPE)) break;
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
-            if (p.qk_norm)
-                rope_norm_tile<BM>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, n0, q_vid, q_pos0, rt, L,
-                                   p);
+            if constexpr (QKN)
+                rope_norm_tile<BM>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, 0u, n0, q_vid, q_pos0,
+                                   rt, L, p);
             else
                 rope_tile<BM>(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
         }
@@ -549,9 +583,9 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int j = 0; j < c.nt; ++j, kr.next()) {
             if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
             const int k0 = c.tile(j) * BN;
-            if (p.qk_norm)
-                rope_norm_tile<BN>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4, k0, k_vid,
-                                   k_pos0, rt, L, p);
+            if constexpr (QKN)
+                rope_norm_tile<BN>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
+                                   p.k_rinv ? sKR + kr.s * KR_BYTES : 0u, k0, k_vid, k_pos0, rt, L, p);
             else if (k0 < k_vid)
                 rope_tile<BN>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
             fence_proxy_async_smem();
@@ -582,7 +616,9 @@ __device__ __forceinline__ uint64_t v_desc_of(uint32_t tile) { return smem_desc_
 // BLOCK: a ring-attention block (Q and K/V rows at their own global offsets,
 // log-sum-exp and optionally fp32 output); the standard call is compiled
 // without that generality (video rows = the first N rows of both, no offsets).
-template <bool BLOCK>
+// QKN: the QK RMSNorm prologue (qk_gamma, qk_eps, optionally k_rinv); a
+// kernel of its own, so that the plain call carries none of its code.
+template <bool BLOCK, bool QKN>
 __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -624,7 +660,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         tmem_relinquish();
     }
     if (p.use_table) build_rope_table(reinterpret_cast<float*>(base_ptr + OFF_TABLE), p);
-    if (p.qk_norm) {
+    if constexpr (QKN) {
         float* gdst = reinterpret_cast<float*>(base_ptr + OFF_GAMMA);
         for (int i = threadIdx.x; i < 4 * D; i += blockDim.x) gdst[i] = __ldg(p.qk_gamma + i);
     }
@@ -639,9 +675,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     const uint32_t sV = sK + static_cast<uint32_t>(p.kstages) * TILE_BYTES;
     const uint32_t sTable = base + OFF_TABLE;
     const uint32_t sGamma = base + OFF_GAMMA;
+    const uint32_t sKR = base + OFF_KR;
 
     if (warp >= WARP_TMA) {
-      regs_decrease<REGS_CONTROL>();
+      regs_decrease<regs_control(QKN)>();
       if (warp == WARP_TMA) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -679,12 +716,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                     // test hook: CTA 0 leaves one K tile unloaded, so that the
                     // next wait for it runs out
                     if (!(p.withhold_k >= 0 && blockIdx.x == 0 && kt == static_cast<uint32_t>(p.withhold_k))) {
-                        mbar_arrive_expect_tx(bar(B_K_FULL + kr.s), TILE_BYTES);
+                        mbar_arrive_expect_tx(bar(B_K_FULL + kr.s), p.k_rinv ? TILE_BYTES + KR_BYTES : TILE_BYTES);
                         armed_k |= 1u << kr.s;
                         par_k = (par_k & ~(1u << kr.s)) | (kr.ph << kr.s);
                         for (int bx = 0; bx < 2; ++bx)
                             tma_load_4d(sK + kr.s * TILE_BYTES + bx * BOX_BYTES, &p.tm_k, bar(B_K_FULL + kr.s),
                                         bx * 64, kc.h, kc.tile(kj) * BN, kc.b);
+                        if (p.k_rinv) {
+                            // the tile's 128 row factors: 512 contiguous bytes, 512-byte aligned
+                            const long long row0 = (static_cast<long long>(kc.b) * p.H + kc.h) * p.k_rinv_ld +
+                                                   static_cast<long long>(kc.tile(kj)) * BN;
+                            bulk_load(sKR + kr.s * KR_BYTES, p.k_rinv + row0, KR_BYTES, bar(B_K_FULL + kr.s));
+                        }
                     }
                     kr.next();
                     ++kt;
@@ -725,7 +768,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
       } else if (warp > WARP_MMA) {
         // RoPE helpers: threads 128..191 of the RoPE role
-        rope_role<BLOCK>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
+        rope_role<BLOCK, QKN>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
@@ -798,9 +841,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
       }
     } else if (warp >= WARP_ROPE) {
-        regs_decrease<REGS_ROPE>();
+        regs_decrease<regs_rope(QKN)>();
         // ------------------------------------------------------------ RoPE
-        rope_role<BLOCK>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma);
+        rope_role<BLOCK, QKN>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -987,8 +1030,8 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
         if (norm) {
             const float* gsrc = (video ? gamma_kv : gamma_kt) + ch0;
             float y[8];
-            rms_norm_chunk(d, __ldg(reinterpret_cast<const float4*>(gsrc)),
-                           __ldg(reinterpret_cast<const float4*>(gsrc + 4)), eps, y);
+            rms_norm_chunk(d, __ldg(reinterpret_cast<const uint4*>(gsrc)),
+                           __ldg(reinterpret_cast<const uint4*>(gsrc + 4)), eps, y);
             uint32_t wv[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -1012,6 +1055,39 @@ __global__ void __launch_bounds__(256) hv_rope_k_kernel(const uint4* __restrict_
             d = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
         if (live) kout[e] = d;
+    }
+}
+
+// Per-row statistics of the QK RMSNorm prologue on load: rinv[(b*H + h)*ld +
+// s] = 1/sqrt(mean_j k_j^2 + eps) for every key row (b, s, h) of K [B, S, H,
+// 128] bf16, by the same arithmetic as rms_norm_chunk (so the attention
+// kernel's normalised keys are bit-identical to those of the two-stage
+// form); the entries s in [S, ld) are set to 0, so that rows past the
+// sequence scale to zero. Memory-bound: reads K once (B*S*H*256 bytes),
+// writes B*H*ld*4 bytes. One half-warp per row, as in hv_rope_k_kernel.
+__global__ void __launch_bounds__(256) hv_k_rinv_kernel(const uint4* __restrict__ kin, float* __restrict__ rinv,
+                                                        long long n_chunks, int H, int S, int ld, float eps) {
+    const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+    const int lane = threadIdx.x & 31;
+    for (long long e0 = static_cast<long long>(blockIdx.x) * blockDim.x + (threadIdx.x - lane); e0 < n_chunks;
+         e0 += step) {
+        const long long e = e0 + lane;
+        const bool live = e < n_chunks;
+        const uint4 d = live ? __ldg(kin + e) : make_uint4(0u, 0u, 0u, 0u);
+        const float r = row_rms_inv(d, eps);
+        if (live && (lane & 15) == 0) {
+            const long long row = e >> 4;   // (b * S + s) * H + h
+            const long long bs = row / H;
+            const int h = static_cast<int>(row - bs * H);
+            const long long b = bs / S;
+            const int s_idx = static_cast<int>(bs - b * S);
+            rinv[(b * H + h) * ld + s_idx] = r;
+        }
+    }
+    const long long n_pad = n_chunks / (16ll * S) * (ld - S);   // B * H * (ld - S)
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_pad; i += step) {
+        const long long bh = i / (ld - S);
+        rinv[bh * ld + S + (i - bh * (ld - S))] = 0.f;
     }
 }
 
@@ -1126,21 +1202,22 @@ static DeviceInfo& device_info(int dev) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         di.sms = sms;
         di.ok = (major == 10 && minor == 0) ? 1 : 0;
-        if (di.ok &&
-            (cudaFuncSetAttribute(hv_attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  SMEM_BYTES) != cudaSuccess ||
-             cudaFuncSetAttribute(hv_attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  SMEM_BYTES) != cudaSuccess))
-            di.ok = 0;
+        const void* kernels[3] = {reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false>)};
+        for (const void* kf : kernels)
+            if (di.ok &&
+                cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+                di.ok = 0;
         // The warpgroups' setmaxnreg split adds up to exactly 512 threads x 128
         // registers; a kernel launched with fewer would wait forever on the
         // increase, so refuse to launch one.
-        const int split = static_cast<int>(2 * 128 * REGS_SOFTMAX + 128 * REGS_ROPE + 128 * REGS_CONTROL);
-        cudaFuncAttributes fa, fb;
-        if (di.ok && (cudaFuncGetAttributes(&fa, hv_attn_fwd_kernel<false>) != cudaSuccess ||
-                      cudaFuncGetAttributes(&fb, hv_attn_fwd_kernel<true>) != cudaSuccess ||
-                      fa.numRegs * NUM_THREADS < split || fb.numRegs * NUM_THREADS < split))
-            di.ok = 0;
+        const int split = static_cast<int>(regs_split(false) > regs_split(true) ? regs_split(false) : regs_split(true));
+        for (const void* kf : kernels) {
+            cudaFuncAttributes fa;
+            if (di.ok && (cudaFuncGetAttributes(&fa, kf) != cudaSuccess || fa.numRegs * NUM_THREADS < split))
+                di.ok = 0;
+        }
     }
     return di;
 }
@@ -1202,6 +1279,8 @@ struct Call {
 // Options of one launch of the attention kernel beyond the call's arguments.
 struct LaunchOpts {
     unsigned long long timeout_ns = kWaitTimeoutNs;
+    const float* k_rinv = nullptr;   // per-row K statistics (QK RMSNorm on load), see Params
+    int k_rinv_ld = 0;
     int withhold_k = -1;   // test hook of hv_attn_selftest_abort
     int h_total = 0;       // heads of the whole call (0: this launch's), for a launch over a head group
     int h_offset = 0;      // first head of the group within the call
@@ -1306,9 +1385,10 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->Wp = Wp;
     prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
     prm->k_rotated = k_rotated ? 1 : 0;
-    prm->qk_norm = qk_gamma != nullptr ? 1 : 0;
     prm->qk_eps = qk_eps;
     prm->qk_gamma = qk_gamma;
+    prm->k_rinv = opts.k_rinv;
+    prm->k_rinv_ld = opts.k_rinv_ld;
     prm->kstages = k_rotated ? KSTAGES_ROTATED : KSTAGES_ROPE;
     prm->vstages = k_rotated ? VSTAGES_ROTATED : VSTAGES_ROPE;
     prm->HpWp = Hp * Wp;
@@ -1338,9 +1418,11 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     // persistent grid: one CTA per SM, at most one per work unit
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
     if (blk)
-        hv_attn_fwd_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+        hv_attn_fwd_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    else if (qk_gamma)
+        hv_attn_fwd_kernel<false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     else
-        hv_attn_fwd_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+        hv_attn_fwd_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     cudaError_t err = cudaSuccess;
     delete prm;
     if (err == cudaSuccess) err = cudaGetLastError();
@@ -1444,8 +1526,32 @@ int hv_attn_forward_qknorm(const void* q, const void* k, const void* v, void* ou
     int st = validate(q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, call, true,
                       qk_gamma, qk_eps);
     if (st != HV_OK) return st;
-    return launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false,
-                            qk_gamma, qk_eps, static_cast<cudaStream_t>(cuda_stream));
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    // 1/rms of every key row, once per call, into stream-ordered scratch
+    // from the device's default memory pool, released behind the attention
+    // kernel on the same stream
+    LaunchOpts opts;
+    opts.k_rinv_ld = (call.S + BN - 1) / BN * BN;
+    const size_t rinv_bytes = static_cast<size_t>(B) * heads * opts.k_rinv_ld * sizeof(float);
+    void* rinv = nullptr;
+    if (cudaMallocAsync(&rinv, rinv_bytes, stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return HV_ERR_LAUNCH;
+    }
+    if (reinterpret_cast<uintptr_t>(rinv) & 15u) {   // the tile copies need 16-byte alignment
+        (void)cudaFreeAsync(rinv, stream);
+        return HV_ERR_LAUNCH;
+    }
+    opts.k_rinv = static_cast<const float*>(rinv);
+    hv_k_rinv_kernel<<<8 * call.sms, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<float*>(rinv),
+                                                       static_cast<long long>(call.bytes / 16), heads, call.S,
+                                                       opts.k_rinv_ld, qk_eps);
+    st = cudaGetLastError() == cudaSuccess ? HV_OK : HV_ERR_LAUNCH;
+    if (st == HV_OK)
+        st = launch_attention(call, q, k, v, out, B, heads, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false,
+                              qk_gamma, qk_eps, stream, nullptr, opts);
+    if (cudaFreeAsync(rinv, stream) != cudaSuccess && st == HV_OK) st = HV_ERR_LAUNCH;
+    return st;
 }
 
 long long hv_attn_workspace_bytes(int B, int heads, int T, int Hp, int Wp, int text_len) {

@@ -112,6 +112,7 @@ def test_qknorm_sampled_parity_720p():
     ((3, 5, 7), 37, [0], False),
     ((5, 3, 11), 100, [1], True),
     ((4, 8, 9), 19, [19, 3, 0], False),
+    ((4, 8, 8), 0, [0], False),          # S = 256: the key statistics need no padding entries
     ((1, 100, 40), 30, [12], False),     # table too large: (cos, sin) per pair
 ])
 def test_qknorm_edge_shapes(grid, text_len, valid, same):
