@@ -363,7 +363,7 @@ def other_workloads(args, dev, stream, peaks):
                  "seq_len": wl.seq_len, "text_valid": tv, "flop_per_call": flops, "steps": steps,
                  "ms_per_call": mean, "ms_min": min(ms), "value": achieved, "unit": UNIT,
                  "frac_of_sustained": achieved / peak, "frac_of_burst": achieved / peak_burst,
-                 "units_512_rows": wl.batch * wl.heads * -(-wl.seq_len // 512), "sms": sms}
+                 "units_256_rows": wl.batch * wl.heads * -(-wl.seq_len // 256), "sms": sms}
         if not args.no_cpu_baseline:
             entry["cpu_baseline"] = cpu_baseline_of(wl, flops, one_core=False)
         res.append(entry)
