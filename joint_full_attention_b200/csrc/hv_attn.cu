@@ -411,7 +411,7 @@ __device__ __forceinline__ void advance8(GridPos& g, const Params& p) {
 // Rows n0 + rb, n0 + rb + 12, ... of a tile of ROWS rows; sequence rows
 // below `vid` are video tokens whose global token index is pos0 + row (the
 // rest are text, left as they are).
-template <int ROWS>
+template <int ROWS, bool TABLE>
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0, int vid, int pos0, int rt,
                                           const RopeLane& L, const Params& p) {
     const int rb = rt >> 4;
@@ -427,7 +427,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
     const uint32_t sin_off = 4u * static_cast<uint32_t>(L.half_dim);
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
     const int stride = 2 * L.half_dim;
-    if (p.use_table) {
+    if constexpr (TABLE) {
         // two rows (r, r + ROPE_GROUPS) per iteration so that their loads overlap
 #pragma unroll 1
         for (int r = rb; r < ROWS; r += 2 * ROPE_GROUPS) {
@@ -486,7 +486,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 // half-warp shuffle: then every lane of a warp runs the same number of
 // iterations (rb and rb + 1 share a warp, and as ROWS is even they share a
 // trip count).
-template <int ROWS>
+template <int ROWS, bool TABLE>
 __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
                                                uint32_t k_rinv, int n0, int vid, int pos0, int rt,
                                                const RopeLane& L, const Params& p) {
@@ -516,7 +516,7 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
             g1 = lds128(gamma_t + gofs + 16);
         }
         uint4 c = make_uint4(0u, 0u, 0u, 0u), sn = c;
-        if (video && p.use_table) {
+        if (TABLE && video) {
             const uint32_t t = tab + 4u * static_cast<uint32_t>(pos * stride);
             c = lds128(t);
             sn = lds128(t + sin_off);
@@ -526,7 +526,7 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
         rms_scale_chunk(d, rr, g0, g1, y);
         uint32_t w[4];
         if (video) {
-            if (p.use_table) {
+            if constexpr (TABLE) {
                 const float cs[4] = {__uint_as_float(c.x), __uint_as_float(c.y), __uint_as_float(c.z),
                                      __uint_as_float(c.w)};
                 const float ss[4] = {__uint_as_float(sn.x), __uint_as_float(sn.y), __uint_as_float(sn.z),
@@ -553,7 +553,7 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
 
 // The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
 // each to the MMA warp.
-template <bool BLOCK, bool QKN>
+template <bool BLOCK, bool QKN, bool TABLE>
 __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
                                           uint32_t sK, uint32_t sTable, uint32_t sGamma, uint32_t sKR) {
     const int q_vid = BLOCK ? p.q_vid : p.N, q_pos0 = BLOCK ? p.q_pos0 : 0;
@@ -570,10 +570,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
             if constexpr (QKN)
-                rope_norm_tile<BM>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, 0u, n0, q_vid, q_pos0,
+                rope_norm_tile<BM, TABLE>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, 0u, n0, q_vid, q_pos0,
                                    rt, L, p);
             else
-                rope_tile<BM>(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
+                rope_tile<BM, TABLE>(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -584,10 +584,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
             if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
             const int k0 = c.tile(j) * BN;
             if constexpr (QKN)
-                rope_norm_tile<BN>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
+                rope_norm_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
                                    p.k_rinv ? sKR + kr.s * KR_BYTES : 0u, k0, k_vid, k_pos0, rt, L, p);
             else if (k0 < k_vid)
-                rope_tile<BN>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
+                rope_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
@@ -618,7 +618,9 @@ __device__ __forceinline__ uint64_t v_desc_of(uint32_t tile) { return smem_desc_
 // without that generality (video rows = the first N rows of both, no offsets).
 // QKN: the QK RMSNorm prologue (qk_gamma, qk_eps, optionally k_rinv); a
 // kernel of its own, so that the plain call carries none of its code.
-template <bool BLOCK, bool QKN>
+// TABLE: (cos, sin) from the shared-memory table (p.use_table = 1), else
+// sincospif per pair; also separate, for the same reason.
+template <bool BLOCK, bool QKN, bool TABLE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -659,7 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
-    if (p.use_table) build_rope_table(reinterpret_cast<float*>(base_ptr + OFF_TABLE), p);
+    if constexpr (TABLE) build_rope_table(reinterpret_cast<float*>(base_ptr + OFF_TABLE), p);
     if constexpr (QKN) {
         float* gdst = reinterpret_cast<float*>(base_ptr + OFF_GAMMA);
         for (int i = threadIdx.x; i < 4 * D; i += blockDim.x) gdst[i] = __ldg(p.qk_gamma + i);
@@ -768,7 +770,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
         }
       } else if (warp > WARP_MMA) {
         // RoPE helpers: threads 128..191 of the RoPE role
-        rope_role<BLOCK, QKN>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
+        rope_role<BLOCK, QKN, TABLE>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
@@ -843,7 +845,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     } else if (warp >= WARP_ROPE) {
         regs_decrease<regs_rope(QKN)>();
         // ------------------------------------------------------------ RoPE
-        rope_role<BLOCK, QKN>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
+        rope_role<BLOCK, QKN, TABLE>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -1202,9 +1204,12 @@ static DeviceInfo& device_info(int dev) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         di.sms = sms;
         di.ok = (major == 10 && minor == 0) ? 1 : 0;
-        const void* kernels[3] = {reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false>)};
+        const void* kernels[6] = {reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false, true>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false, false>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true, true>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true, false>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false, true>),
+                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false, false>)};
         for (const void* kf : kernels)
             if (di.ok &&
                 cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
@@ -1418,11 +1423,14 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     // persistent grid: one CTA per SM, at most one per work unit
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
     if (blk)
-        hv_attn_fwd_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+        (prm->use_table ? hv_attn_fwd_kernel<true, false, true> : hv_attn_fwd_kernel<true, false, false>)
+            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     else if (qk_gamma)
-        hv_attn_fwd_kernel<false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+        (prm->use_table ? hv_attn_fwd_kernel<false, true, true> : hv_attn_fwd_kernel<false, true, false>)
+            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     else
-        hv_attn_fwd_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+        (prm->use_table ? hv_attn_fwd_kernel<false, false, true> : hv_attn_fwd_kernel<false, false, false>)
+            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     cudaError_t err = cudaSuccess;
     delete prm;
     if (err == cudaSuccess) err = cudaGetLastError();
