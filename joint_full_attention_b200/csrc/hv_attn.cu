@@ -137,7 +137,6 @@ struct __align__(64) Params {
     void* out;          // bf16 [B, S, H, 128], or fp32 when out_f32
     int B, H, S, N, T, Hp, Wp, HpWp;
     int use_table;      // 1: cos/sin from the shared-memory table, 0: sincospif per pair
-    int k_rotated;      // 1: K already holds rotated keys (workspace path): rotate Q only
     float qk_eps;       // RMSNorm epsilon
     const float* qk_gamma;   // device, fp32 [4][128]: Q video, K video, Q text, K text
     // Optional, with the QK RMSNorm: 1/rms of every K row, fp32 [B, H, k_rinv_ld]
@@ -147,8 +146,6 @@ struct __align__(64) Params {
     // every row again for every unit.
     const float* k_rinv;
     int k_rinv_ld;
-    int kstages;        // K tiles in flight (slots 0 .. kstages-1 of the KV pool)
-    int vstages;        // V tiles in flight (the next vstages slots)
     int n_qunits;       // ceil(S / 256)
     int units;          // B * H * n_qunits
     float theta_log2;   // log2(rope_theta)
@@ -217,11 +214,15 @@ struct Waiter {
 
 // Position in a ring of n stages: the stage in use and the parity of its
 // current fill (flips each time the ring wraps).
+// Cursor over a ring of N stages: stage s, and the mbarrier phase parity of
+// the current pass over the ring.
+template <uint32_t N>
 struct Ring {
-    uint32_t n, s, ph;
-    __device__ __forceinline__ explicit Ring(int stages) : n(static_cast<uint32_t>(stages)), s(0), ph(0) {}
+    uint32_t s = 0, ph = 0;
     __device__ __forceinline__ void next() {
-        if (++s == n) {
+        if constexpr (N == 1) {
+            ph ^= 1u;
+        } else if (++s == N) {
             s = 0;
             ph ^= 1u;
         }
@@ -553,7 +554,7 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
 
 // The RoPE role: rotate the Q tiles of every unit and every K tile, then hand
 // each to the MMA warp.
-template <bool BLOCK, bool QKN, bool TABLE>
+template <bool BLOCK, bool QKN, bool KROT, bool TABLE>
 __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter& waiter, uint32_t bars, uint32_t sQ,
                                           uint32_t sK, uint32_t sTable, uint32_t sGamma, uint32_t sKR) {
     const int q_vid = BLOCK ? p.q_vid : p.N, q_pos0 = BLOCK ? p.q_pos0 : 0;
@@ -561,7 +562,7 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
     const RopeLane L = make_rope_lane(rt, p);
     const int lane = threadIdx.x & 31;
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-    Ring kr(p.kstages);
+    Ring<KSTAGES_ROPE> kr;
     uint32_t lu = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
         const UnitCoord c = decode_unit(p, u);
@@ -579,7 +580,7 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_Q_READY));
         bool ok = true;
-        if (p.k_rotated) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
+        if constexpr (KROT) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
         for (int j = 0; j < c.nt; ++j, kr.next()) {
             if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
             const int k0 = c.tile(j) * BN;
@@ -618,9 +619,11 @@ __device__ __forceinline__ uint64_t v_desc_of(uint32_t tile) { return smem_desc_
 // without that generality (video rows = the first N rows of both, no offsets).
 // QKN: the QK RMSNorm prologue (qk_gamma, qk_eps, optionally k_rinv); a
 // kernel of its own, so that the plain call carries none of its code.
-// TABLE: (cos, sin) from the shared-memory table (p.use_table = 1), else
-// sincospif per pair; also separate, for the same reason.
-template <bool BLOCK, bool QKN, bool TABLE>
+// KROT: K holds rotated keys (workspace paths): the RoPE warps rotate Q only
+// and the K/V ring is split 2 + 2 instead of 3 + 1. TABLE: (cos, sin) from
+// the shared-memory table (p.use_table = 1), else sincospif per pair. Each a
+// kernel of its own, for the same reason.
+template <bool BLOCK, bool QKN, bool KROT, bool TABLE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -674,7 +677,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     const Waiter waiter{abort_flag, p.timeout_ns, p.status};
     const uint32_t sQ = base + OFF_Q;
     const uint32_t sK = base + OFF_KV;
-    const uint32_t sV = sK + static_cast<uint32_t>(p.kstages) * TILE_BYTES;
+    constexpr int KST = KROT ? KSTAGES_ROTATED : KSTAGES_ROPE;
+    constexpr int VST = KROT ? VSTAGES_ROTATED : VSTAGES_ROPE;
+    const uint32_t sV = sK + static_cast<uint32_t>(KST) * TILE_BYTES;
     const uint32_t sTable = base + OFF_TABLE;
     const uint32_t sGamma = base + OFF_GAMMA;
     const uint32_t sKR = base + OFF_KR;
@@ -690,7 +695,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             // Two cursors over this CTA's (unit, tile) sequence: keys (each
             // unit's Q ahead of its first key) run up to kstages tiles ahead
             // of the values.
-            Ring kr(p.kstages), vr(p.vstages);
+            Ring<KST> kr;
+            Ring<VST> vr;
             uint32_t kt = 0, vt = 0, klu = 0;   // K and V tiles issued, units whose Q is issued
             int ku = blockIdx.x, kj = 0, vu = blockIdx.x, vj = 0;
             UnitCoord kc{}, vc{};
@@ -700,7 +706,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             uint32_t par_q = 0, par_k = 0, par_v = 0;
             bool ok = true;
             while (ok && vu < p.units) {
-                while (ku < p.units && kt < vt + kr.n) {
+                while (ku < p.units && kt < vt + KST) {
                     if (kj == 0) {
                         // The Q buffer frees when the previous unit's last QK
                         // MMA completes, which needs that unit's values up to
@@ -762,28 +768,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 volatile int never = 0;
                 Waiter tail{&never, 20000000ull, nullptr, false};
                 if (armed_q) tail.wait(bar(B_Q_FULL), par_q, ROLE_TMA);
-                for (int s = 0; s < p.kstages; ++s)
+                for (int s = 0; s < KST; ++s)
                     if ((armed_k >> s) & 1u) tail.wait(bar(B_K_FULL + s), (par_k >> s) & 1u, ROLE_TMA);
-                for (int s = 0; s < p.vstages; ++s)
+                for (int s = 0; s < VST; ++s)
                     if ((armed_v >> s) & 1u) tail.wait(bar(B_V_FULL + s), (par_v >> s) & 1u, ROLE_TMA);
             }
         }
       } else if (warp > WARP_MMA) {
         // RoPE helpers: threads 128..191 of the RoPE role
-        rope_role<BLOCK, QKN, TABLE>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
+        rope_role<BLOCK, QKN, KROT, TABLE>(128 + threadIdx.x - (WARP_MMA + 1) * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
       } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
             // K tiles are ready for the tensor core once the RoPE warps have
             // rotated them, or, when they arrive rotated, once TMA lands them.
-            const int k_ready = p.k_rotated ? B_K_FULL : B_K_READY;
+            constexpr int k_ready = KROT ? B_K_FULL : B_K_READY;
             // operand descriptors, computed once: the MMAs only add offsets
             // (a stage's tile lies TILE_BYTES / 16 address units after the previous one)
             const uint64_t dq0 = kmajor_desc(sQ), dq1 = kmajor_desc(sQ + TILE_BYTES);
             const uint64_t dk0 = kmajor_desc(sK), dv0 = v_desc_of(sV);
             auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (TILE_BYTES / 16)); };
             auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (TILE_BYTES / 16)); };
-            Ring kr(p.kstages), vr(p.vstages);
+            Ring<KST> kr;
+            Ring<VST> vr;
             uint32_t lu = 0;
             uint32_t pr[QTILES] = {0, 0};
             bool ok = true;
@@ -845,7 +852,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
     } else if (warp >= WARP_ROPE) {
         regs_decrease<regs_rope(QKN)>();
         // ------------------------------------------------------------ RoPE
-        rope_role<BLOCK, QKN, TABLE>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
+        rope_role<BLOCK, QKN, KROT, TABLE>(threadIdx.x - WARP_ROPE * 32, p, waiter, bars, sQ, sK, sTable, sGamma, sKR);
     } else {
         regs_increase<REGS_SOFTMAX>();
         // --------------------------------------------------------- softmax
@@ -1192,6 +1199,35 @@ struct DeviceInfo {
     int sms = 0;
 };
 
+// The attention kernel's instantiations: a ring-attention block (plain keys
+// only), or the standard call with or without the QK RMSNorm prologue and
+// with or without pre-rotated keys; each with and without the rotation table.
+using AttnKernel = void (*)(Params);
+
+template <bool BLOCK, bool QKN, bool KROT>
+static AttnKernel attn_kernel(bool table) {
+    return table ? hv_attn_fwd_kernel<BLOCK, QKN, KROT, true> : hv_attn_fwd_kernel<BLOCK, QKN, KROT, false>;
+}
+
+static AttnKernel kernel_for(bool block, bool qkn, bool krot, bool table) {
+    if (block) return attn_kernel<true, false, false>(table);
+    if (qkn) return krot ? attn_kernel<false, true, true>(table) : attn_kernel<false, true, false>(table);
+    return krot ? attn_kernel<false, false, true>(table) : attn_kernel<false, false, false>(table);
+}
+
+// Every instantiation, for the per-device set-up.
+constexpr int N_KERNELS = 10;
+static AttnKernel kernel_at(int i) {
+    const bool table = i & 1;
+    switch (i >> 1) {
+        case 0: return kernel_for(false, false, false, table);
+        case 1: return kernel_for(false, false, true, table);
+        case 2: return kernel_for(false, true, false, table);
+        case 3: return kernel_for(false, true, true, table);
+        default: return kernel_for(true, false, false, table);
+    }
+}
+
 static DeviceInfo& device_info(int dev) {
     static DeviceInfo infos[64];
     static std::mutex mu;
@@ -1204,12 +1240,8 @@ static DeviceInfo& device_info(int dev) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         di.sms = sms;
         di.ok = (major == 10 && minor == 0) ? 1 : 0;
-        const void* kernels[6] = {reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false, true>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, false, false>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true, true>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<false, true, false>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false, true>),
-                                  reinterpret_cast<const void*>(hv_attn_fwd_kernel<true, false, false>)};
+        const void* kernels[N_KERNELS];
+        for (int i = 0; i < N_KERNELS; ++i) kernels[i] = reinterpret_cast<const void*>(kernel_at(i));
         for (const void* kf : kernels)
             if (di.ok &&
                 cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
@@ -1389,13 +1421,10 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     prm->Hp = Hp;
     prm->Wp = Wp;
     prm->use_table = (8ll * T + 28ll * (Hp + static_cast<long long>(Wp))) <= TABLE_MAX_ENTRIES ? 1 : 0;
-    prm->k_rotated = k_rotated ? 1 : 0;
     prm->qk_eps = qk_eps;
     prm->qk_gamma = qk_gamma;
     prm->k_rinv = opts.k_rinv;
     prm->k_rinv_ld = opts.k_rinv_ld;
-    prm->kstages = k_rotated ? KSTAGES_ROTATED : KSTAGES_ROPE;
-    prm->vstages = k_rotated ? VSTAGES_ROTATED : VSTAGES_ROPE;
     prm->HpWp = Hp * Wp;
     prm->n_qunits = (S + UNIT_ROWS - 1) / UNIT_ROWS;
     prm->units = static_cast<int>(call.units);
@@ -1422,15 +1451,8 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     }
     // persistent grid: one CTA per SM, at most one per work unit
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
-    if (blk)
-        (prm->use_table ? hv_attn_fwd_kernel<true, false, true> : hv_attn_fwd_kernel<true, false, false>)
-            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
-    else if (qk_gamma)
-        (prm->use_table ? hv_attn_fwd_kernel<false, true, true> : hv_attn_fwd_kernel<false, true, false>)
-            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
-    else
-        (prm->use_table ? hv_attn_fwd_kernel<false, false, true> : hv_attn_fwd_kernel<false, false, false>)
-            <<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
+    const AttnKernel kern = kernel_for(blk != nullptr, qk_gamma != nullptr, k_rotated, prm->use_table != 0);
+    kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     cudaError_t err = cudaSuccess;
     delete prm;
     if (err == cudaSuccess) err = cudaGetLastError();
