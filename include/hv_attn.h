@@ -336,8 +336,10 @@ int hv_attn_selftest_timeout(int timeout_us);
  * rotated on load, rope_theta 256, scale 1/sqrt(128)) on the caller's problem
  * with every wait bounded by timeout_us microseconds (1000..1000000) and with
  * CTA 0 leaving its K tile load number withhold_k (>= 0, counted over that
- * CTA's loads) unissued, so that the wait of its RoPE warps for those keys
- * runs out. That CTA then stops every role, lets its copies and MMAs in
+ * CTA's loads) unissued, so that a wait runs out: the RoPE warps' for those
+ * keys, or the producer's for the stage they hold (whichever polls first
+ * past the limit records its role). That CTA then stops every role, lets
+ * its copies and MMAs in
  * flight finish, frees its TMEM and returns, while the other CTAs finish. Synchronises `cuda_stream`, then returns HV_OK;
  * the error word and the host status word are set as for any timeout (read
  * and clear them with hv_attn_last_device_error). `out` is left partly
