@@ -212,27 +212,34 @@ int hv_attn_forward_noalloc(const void* q, const void* k, const void* v, void* o
 /*
  * hv_attn_forward_host - the whole call from and to HOST memory, with the
  * copies overlapping the attention kernel. The heads are cut into
- * `head_groups` groups (heads % head_groups == 0); per group, in a pipeline
- * of two device staging slots: a 2-D copy of the group's q, k, v columns
- * host -> device, hv_attn_forward on the contiguous [B, S, heads/groups, 128]
- * staging tensors, and a 2-D copy of the group's output columns back into
- * out_host. Heads are independent (§5.2 computes attention per head), so the
- * result equals hv_attn_forward's bit for bit. No counterpart in the pages:
- * it is the host-buffer form of the same call.
+ * `head_groups` groups (heads % head_groups == 0), and the first and the
+ * last group further into one head and the rest, so that only one head's
+ * columns are copied in before the first kernel and out after the last.
+ * Per piece, in a pipeline of two device staging slots: a 2-D copy of the
+ * piece's q, k, v columns host -> device, the attention kernel on the
+ * contiguous [B, S, heads_of_piece, 128] staging tensors, and a 2-D copy of
+ * its output columns back into out_host. The kernels of consecutive pieces
+ * alternate between two streams, so that one piece's kernel takes the SMs
+ * the previous one frees during its last wave. Heads are independent (§5.2
+ * computes attention per head), so the result equals hv_attn_forward's bit
+ * for bit. No counterpart in the pages: it is the host-buffer form of the
+ * same call.
  *
  * q_host, k_host, v_host, out_host: HOST pointers, layout as hv_attn_forward;
  *            page-locked (pinned) memory lets the copies run asynchronously;
  *            out_host must not overlap the inputs.
- * head_groups: >= 1, dividing heads (1 = no overlap, copies and compute in turn).
+ * head_groups: >= 1, dividing heads.
  * workspace: DEVICE pointer, 16-byte aligned, at least
  *            hv_attn_host_workspace_bytes(...) bytes, owned by the caller.
- * cuda_stream: the kernels run on it; the copies run on two streams the
- *            library creates once per device (make the first call before any
- *            stream capture). The call is asynchronous: `cuda_stream` is made to
- *            wait for the last copy, so out_host is complete once that stream
- *            has been synchronised; the host buffers must stay valid until then.
- *            Calls on one device share the copy streams and are enqueued one
- *            at a time (a mutex), so they run in turn.
+ * cuda_stream: the copies and kernels run on four streams the library
+ *            creates once per device (copies in, copies out, two for the
+ *            kernels; make the first call before any stream capture), ordered
+ *            after the work already enqueued on `cuda_stream`. The call is
+ *            asynchronous: `cuda_stream` is made to wait for the last copy, so
+ *            out_host is complete once that stream has been synchronised; the
+ *            host buffers must stay valid until then. Calls on one device
+ *            share these streams and are enqueued one at a time (a mutex), so
+ *            they run in turn.
  * Errors: HV_ERR_NULL_POINTER, HV_ERR_BAD_SHAPE (also bad head_groups),
  * HV_ERR_BAD_TEXT, HV_ERR_ALIAS (host buffers), HV_ERR_WORKSPACE, and those of
  * hv_attn_forward for one group's call; HV_ERR_LAUNCH if a copy or a stream

@@ -579,21 +579,23 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_Q_READY));
-        bool ok = true;
-        if constexpr (KROT) continue;   // keys arrive rotated: the MMA warp takes them straight from TMA
-        for (int j = 0; j < c.nt; ++j, kr.next()) {
-            if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
-            const int k0 = c.tile(j) * BN;
-            if constexpr (QKN)
-                rope_norm_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
-                                   p.k_rinv ? sKR + kr.s * KR_BYTES : 0u, k0, k_vid, k_pos0, rt, L, p);
-            else if (k0 < k_vid)
-                rope_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
+        // with KROT the keys arrive rotated: the MMA warp takes them straight from TMA
+        if constexpr (!KROT) {
+            bool ok = true;
+            for (int j = 0; j < c.nt; ++j, kr.next()) {
+                if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
+                const int k0 = c.tile(j) * BN;
+                if constexpr (QKN)
+                    rope_norm_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
+                                              p.k_rinv ? sKR + kr.s * KR_BYTES : 0u, k0, k_vid, k_pos0, rt, L, p);
+                else if (k0 < k_vid)
+                    rope_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_K_READY + kr.s));
+            }
+            if (!ok) break;
         }
-        if (!ok) break;
     }
 }
 
@@ -1472,9 +1474,14 @@ static int launch_rope_k(const Call& call, const void* k, void* dst, int heads, 
 }
 
 // Streams and events of the host-buffer pipeline, created once per device.
+// Streams and events of the host-buffer pipeline, per device: copies in and
+// out on their own streams, and the attention launches alternating between
+// two compute streams, so that a launch's CTAs take the SMs the previous
+// launch's CTAs leave while its last wave finishes (independent heads, no
+// kernel waits on another).
 struct HostPipe {
     bool ok = false;
-    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaStream_t h2d = nullptr, d2h = nullptr, comp[2] = {};
     cudaEvent_t start = nullptr;
     cudaEvent_t h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
 };
@@ -1487,6 +1494,8 @@ static HostPipe* host_pipe(int dev) {
     if (!hp.ok) {
         bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
                     cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.comp[0], cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.comp[1], cudaStreamNonBlocking) == cudaSuccess &&
                     cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
         for (int i = 0; i < 2 && good; ++i)
             good = cudaEventCreateWithFlags(&hp.h2d_done[i], cudaEventDisableTiming) == cudaSuccess &&
@@ -1681,40 +1690,63 @@ int hv_attn_forward_host(const void* q_host, const void* k_host, const void* v_h
     HostPipe* hp = host_pipe(dev);
     if (!hp) return HV_ERR_LAUNCH;
     const cudaStream_t cs = static_cast<cudaStream_t>(cuda_stream);
-    const size_t row = static_cast<size_t>(heads) * D * 2, grow = static_cast<size_t>(hg) * D * 2;
+    const size_t row = static_cast<size_t>(heads) * D * 2;
     const size_t rows = static_cast<size_t>(B) * call.S;
     bool good = cudaEventRecord(hp->start, cs) == cudaSuccess &&
                 cudaStreamWaitEvent(hp->h2d, hp->start, 0) == cudaSuccess &&
-                cudaStreamWaitEvent(hp->d2h, hp->start, 0) == cudaSuccess;
+                cudaStreamWaitEvent(hp->d2h, hp->start, 0) == cudaSuccess &&
+                cudaStreamWaitEvent(hp->comp[0], hp->start, 0) == cudaSuccess &&
+                cudaStreamWaitEvent(hp->comp[1], hp->start, 0) == cudaSuccess;
     const void* src[3] = {q_host, k_host, v_host};
-    for (int g = 0; g < head_groups && good; ++g) {
-        const int slot = g & 1;
-        const size_t col = static_cast<size_t>(g) * grow;
-        // inputs of this group into the slot, once the group that used it last has been computed
-        good = cudaStreamWaitEvent(hp->h2d, hp->comp_done[slot], 0) == cudaSuccess;
+    int piece = 0;   // pieces enqueued so far; piece i uses slot i & 1 and compute stream i & 1
+    // One piece: heads h0 .. h0 + n - 1 copied in, computed and copied out.
+    auto run_piece = [&](int h0, int n) {
+        const int slot = piece++ & 1;
+        const cudaStream_t comp = hp->comp[slot];
+        const size_t col = static_cast<size_t>(h0) * D * 2, grow = static_cast<size_t>(n) * D * 2;
+        // inputs of this piece into the slot, once the piece that used it last has been computed
+        good = good && cudaStreamWaitEvent(hp->h2d, hp->comp_done[slot], 0) == cudaSuccess;
         for (int t = 0; t < 3 && good; ++t)
             good = cudaMemcpy2DAsync(slot_buf(slot, t), grow, static_cast<const uint8_t*>(src[t]) + col, row, grow,
                                      rows, cudaMemcpyHostToDevice, hp->h2d) == cudaSuccess;
         good = good && cudaEventRecord(hp->h2d_done[slot], hp->h2d) == cudaSuccess;
-        // attention of the group, once its inputs are in and the slot's output has been copied out
-        good = good && cudaStreamWaitEvent(cs, hp->h2d_done[slot], 0) == cudaSuccess &&
-               cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
+        // attention of the piece, once its inputs are in and the slot's output has been copied out
+        good = good && cudaStreamWaitEvent(comp, hp->h2d_done[slot], 0) == cudaSuccess &&
+               cudaStreamWaitEvent(comp, hp->d2h_done[slot], 0) == cudaSuccess;
         if (good) {
+            Call pc = call;
+            pc.units = static_cast<long long>(B) * n * ((call.S + UNIT_ROWS - 1) / UNIT_ROWS);
             LaunchOpts opts;
             opts.h_total = heads;
-            opts.h_offset = g * hg;
-            st = launch_attention(call, slot_buf(slot, 0), slot_buf(slot, 1), slot_buf(slot, 2), slot_buf(slot, 3), B,
-                                  hg, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false, nullptr, 0.f, cs,
+            opts.h_offset = h0;
+            st = launch_attention(pc, slot_buf(slot, 0), slot_buf(slot, 1), slot_buf(slot, 2), slot_buf(slot, 3), B,
+                                  n, T, Hp, Wp, text_len, text_valid, rope_theta, scale, false, nullptr, 0.f, comp,
                                   nullptr, opts);
-            if (st != HV_OK) return st;
+            if (st != HV_OK) good = false;
         }
-        good = good && cudaEventRecord(hp->comp_done[slot], cs) == cudaSuccess;
-        // the group's output back into its columns of out_host
+        good = good && cudaEventRecord(hp->comp_done[slot], comp) == cudaSuccess;
+        // the piece's output back into its columns of out_host
         good = good && cudaStreamWaitEvent(hp->d2h, hp->comp_done[slot], 0) == cudaSuccess &&
                cudaMemcpy2DAsync(static_cast<uint8_t*>(out_host) + col, row, slot_buf(slot, 3), grow, grow, rows,
                                  cudaMemcpyDeviceToHost, hp->d2h) == cudaSuccess &&
                cudaEventRecord(hp->d2h_done[slot], hp->d2h) == cudaSuccess;
+    };
+    // The head groups in order; the first and the last are cut into one head
+    // and the rest, so that only one head's columns are copied in before the
+    // first kernel and copied out after the last.
+    for (int g = 0; g < head_groups && good; ++g) {
+        const int h0 = g * hg;
+        if (hg > 1 && g == 0) {
+            run_piece(h0, 1);
+            run_piece(h0 + 1, hg - 1);
+        } else if (hg > 1 && g == head_groups - 1) {
+            run_piece(h0, hg - 1);
+            run_piece(h0 + hg - 1, 1);
+        } else {
+            run_piece(h0, hg);
+        }
     }
+    if (st != HV_OK) return st;
     // the caller's stream completes after the last copy out
     for (int slot = 0; slot < 2 && good; ++slot) good = cudaStreamWaitEvent(cs, hp->d2h_done[slot], 0) == cudaSuccess;
     return good ? HV_OK : HV_ERR_LAUNCH;
