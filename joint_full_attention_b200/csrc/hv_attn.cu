@@ -694,6 +694,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             tma_prefetch_desc(&p.tm_q);
             tma_prefetch_desc(&p.tm_k);
             tma_prefetch_desc(&p.tm_v);
+            // Q tiles are read once per call: evicted from L2 first, so that
+            // the K/V tiles every unit re-reads stay there longer
+            const uint64_t once = l2_evict_first_policy();
             // Two cursors over this CTA's (unit, tile) sequence: keys (each
             // unit's Q ahead of its first key) run up to kstages tiles ahead
             // of the values.
@@ -719,8 +722,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                         armed_q = 1; par_q = klu & 1;
                         for (int qi = 0; qi < QTILES; ++qi)
                             for (int bx = 0; bx < 2; ++bx)
-                                tma_load_4d(sQ + qi * TILE_BYTES + bx * BOX_BYTES, &p.tm_q, bar(B_Q_FULL), bx * 64,
-                                            kc.h, kc.qu * UNIT_ROWS + qi * BM, kc.b);
+                                tma_load_4d_hint(sQ + qi * TILE_BYTES + bx * BOX_BYTES, &p.tm_q, bar(B_Q_FULL),
+                                                 bx * 64, kc.h, kc.qu * UNIT_ROWS + qi * BM, kc.b, once);
                     }
                     if (!(ok = waiter.wait(bar(B_K_EMPTY + kr.s), kr.ph ^ 1, ROLE_TMA))) break;
                     // test hook: CTA 0 leaves one K tile unloaded, so that the
@@ -977,6 +980,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 }
             }
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D);
+            const uint64_t once = l2_evict_first_policy();   // output rows: written once, evicted first
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t r[32];
@@ -990,7 +994,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
                 if (store) {
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4)
-                        dst[ch * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                        stg128_hint(dst + ch * 4 + v4,
+                                    make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]), once);
                 }
             }
             tc_fence_before();
