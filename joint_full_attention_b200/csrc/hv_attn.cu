@@ -48,10 +48,10 @@ constexpr int BN = 128;             // keys per K/V tile
 constexpr int QTILES = 2;           // Q tiles per work unit
 constexpr int UNIT_ROWS = BM * QTILES;
 // K and V tiles share a pool of KV_SLOTS shared-memory tiles: K takes the
-// first kstages slots and V the next vstages (chosen per launch). When the
-// RoPE warps rotate K, three K stages and one V stage let them work on K tiles
-// up to two tiles ahead of the tensor core; pre-rotated keys need no lead and
-// keep two of each.
+// first KST slots and V the next VST (fixed per kernel instantiation). When
+// the RoPE warps rotate K, three K stages and one V stage let them work on K
+// tiles up to two tiles ahead of the tensor core; pre-rotated keys need no
+// lead and keep two of each.
 constexpr int KV_SLOTS = 4;
 constexpr int KSTAGES_MAX = 3;
 constexpr int VSTAGES_MAX = 2;
@@ -698,7 +698,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) hv_attn_fwd_kernel(const __gri
             // the K/V tiles every unit re-reads stay there longer
             const uint64_t once = l2_evict_first_policy();
             // Two cursors over this CTA's (unit, tile) sequence: keys (each
-            // unit's Q ahead of its first key) run up to kstages tiles ahead
+            // unit's Q ahead of its first key) run up to KST tiles ahead
             // of the values.
             Ring<KST> kr;
             Ring<VST> vr;
