@@ -340,3 +340,22 @@ def test_host_pipeline_bit_identical(name, groups, pinned):
         out = H.attn_forward_host(*host, wl.grid, wl.text_len, inp["text_valid"], work=work, head_groups=groups)
         assert torch.equal(out, ref)
     assert H.last_device_error() == 0
+
+
+@pytest.mark.parametrize("heads,groups", [(1, 1), (2, 1), (3, 1), (2, 2), (4, 2), (6, 3)])
+def test_host_pipeline_pieces(heads, groups):
+    """The pipeline's pieces: the first and the last head group are cut into one
+    head and the rest (a single group of 2 or 3 heads becomes 1 + 1 or 1 + 2;
+    groups of one head are not cut), alternating slots and kernel streams.
+    Every split returns what hv_attn_forward computes, bit for bit, on a
+    batch of two samples with different valid text lengths."""
+    wl = W.Workload("pieces", "pieces", 2, heads, (2, 6, 5), 7, valid=(7, 3))
+    inp = W.make_inputs(wl, seed=8)
+    q, k, v = (to_dev(inp[n]) for n in ("q", "k", "v"))
+    ref = H.attn_forward(q, k, v, wl.grid, wl.text_len, inp["text_valid"]).cpu()
+    host = [torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")]
+    work = {}
+    for _ in range(2):
+        out = H.attn_forward_host(*host, wl.grid, wl.text_len, inp["text_valid"], work=work, head_groups=groups)
+        assert torch.equal(out, ref)
+    assert H.last_device_error() == 0
