@@ -481,13 +481,13 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
 // tile of ROWS rows (rows rb, rb + 12, ...); text rows and rows past the
 // sequence are only normalised (rows past the sequence hold TMA's zero fill
 // and stay zero). gamma_v / gamma_t: shared-memory addresses of the video /
-// text gamma of this tensor (Q or K). k_rinv: shared-memory address of the
-// tile's 128 row factors 1/rms when they were computed beforehand (K tiles
-// with per-row statistics), else 0 and each row's sum is reduced here, a
-// half-warp shuffle: then every lane of a warp runs the same number of
-// iterations (rb and rb + 1 share a warp, and as ROWS is even they share a
-// trip count).
-template <int ROWS, bool TABLE>
+// text gamma of this tensor (Q or K). RINV: the tile's 128 row factors 1/rms
+// were computed beforehand and sit at shared-memory address k_rinv (K tiles);
+// otherwise each row's sum is reduced here, a half-warp shuffle, and every
+// lane of a warp runs the same number of iterations (rb and rb + 1 share a
+// warp, and as ROWS is even they share a trip count). Separate
+// instantiations keep each call site's code to the one it uses.
+template <int ROWS, bool TABLE, bool RINV>
 __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, uint32_t gamma_v, uint32_t gamma_t,
                                                uint32_t k_rinv, int n0, int vid, int pos0, int rt,
                                                const RopeLane& L, const Params& p) {
@@ -523,7 +523,11 @@ __device__ __forceinline__ void rope_norm_tile(uint32_t tile, uint32_t table, ui
             sn = lds128(t + sin_off);
         }
         float y[8];
-        const float rr = k_rinv ? lds_f32(k_rinv + 4u * static_cast<uint32_t>(r)) : row_rms_inv(d, p.qk_eps);
+        float rr;
+        if constexpr (RINV)
+            rr = lds_f32(k_rinv + 4u * static_cast<uint32_t>(r));
+        else
+            rr = row_rms_inv(d, p.qk_eps);
         rms_scale_chunk(d, rr, g0, g1, y);
         uint32_t w[4];
         if (video) {
@@ -571,7 +575,7 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
         for (int qi = 0; qi < QTILES; ++qi) {
             const int n0 = c.qu * UNIT_ROWS + qi * BM;
             if constexpr (QKN)
-                rope_norm_tile<BM, TABLE>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, 0u, n0, q_vid, q_pos0,
+                rope_norm_tile<BM, TABLE, false>(sQ + qi * TILE_BYTES, sTable, sGamma, sGamma + 2 * D * 4, 0u, n0, q_vid, q_pos0,
                                    rt, L, p);
             else
                 rope_tile<BM, TABLE>(sQ + qi * TILE_BYTES, sTable, n0, q_vid, q_pos0, rt, L, p);
@@ -585,9 +589,10 @@ __device__ __forceinline__ void rope_role(int rt, const Params& p, const Waiter&
             for (int j = 0; j < c.nt; ++j, kr.next()) {
                 if (!(ok = waiter.wait(bar(B_K_FULL + kr.s), kr.ph, ROLE_ROPE))) break;
                 const int k0 = c.tile(j) * BN;
-                if constexpr (QKN)
-                    rope_norm_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4, sGamma + 3 * D * 4,
-                                              p.k_rinv ? sKR + kr.s * KR_BYTES : 0u, k0, k_vid, k_pos0, rt, L, p);
+                if constexpr (QKN)   // keys normalised on load always come with their row factors
+                    rope_norm_tile<BN, TABLE, true>(sK + kr.s * TILE_BYTES, sTable, sGamma + D * 4,
+                                                    sGamma + 3 * D * 4, sKR + kr.s * KR_BYTES, k0, k_vid, k_pos0,
+                                                    rt, L, p);
                 else if (k0 < k_vid)
                     rope_tile<BN, TABLE>(sK + kr.s * TILE_BYTES, sTable, k0, k_vid, k_pos0, rt, L, p);
                 fence_proxy_async_smem();
@@ -1458,6 +1463,11 @@ static int launch_attention(const Call& call, const void* q, const void* k, cons
     }
     // persistent grid: one CTA per SM, at most one per work unit
     const int grid = static_cast<int>(call.units < call.sms ? call.units : call.sms);
+    // keys normalised on load always come with their row factors (hv_k_rinv_kernel)
+    if (qk_gamma != nullptr && !k_rotated && opts.k_rinv == nullptr) {
+        delete prm;
+        return HV_ERR_LAUNCH;
+    }
     const AttnKernel kern = kernel_for(blk != nullptr, qk_gamma != nullptr, k_rotated, prm->use_table != 0);
     kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(*prm);
     cudaError_t err = cudaSuccess;
