@@ -118,9 +118,10 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_per_launch():
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
-    if not TRAFFIC_SUMMARY.exists():
+def traffic_per_launch(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it covers this
+    workload and matches this source."""
+    if not TRAFFIC_SUMMARY.exists() or f".{workload}." not in TRAFFIC_SUMMARY.name:
         return None
     text = TRAFFIC_SUMMARY.read_text()
     m_src = re.search(r"source_digest:\s*([0-9a-f]+)", text)
@@ -511,7 +512,7 @@ def run_ours(args, wl, inp, rank, world, local):
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-        "traffic": traffic_per_launch(), "kernel": KERNEL_NAME,
+        "traffic": traffic_per_launch(args.workload), "kernel": KERNEL_NAME,
         "peak_source": f"bf16_tflops_sustained of {peak_kind} (cuBLAS bf16 loop under the power cap); "
                        "the step is a seconds-long loop of one kernel",
         "frac_of_burst": achieved / peak_burst, "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
