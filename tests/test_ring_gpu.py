@@ -86,6 +86,34 @@ def test_whole_sequence_block_is_the_plain_call():
     assert o32.dtype == torch.float32 and torch.equal(o32.to(torch.bfloat16), ref)
 
 
+def test_block_on_grid_without_table():
+    """A grid whose rotation table would not fit in shared memory (8*T' + 28*(H'/2 + W'/2) = 3928
+    entries against 3840): the block kernel's per-pair sincospif form, against the oracle at run
+    offsets, and over the whole sequence equal to the plain call (which takes the same form)."""
+    grid = (1, 100, 40)                                 # 4000 video tokens
+    heads = 2
+    sq, q_video, q_pos0, sk, k_video, k_pos0, kv = 240, 200, 3700, 300, 300, 100, [300]
+    qb, kb, vb = _bits((1, sq, heads, 128), 11), _bits((1, sk, heads, 128), 12), _bits((1, sk, heads, 128), 13)
+    o, lse = H.attn_forward_block(_dev(qb), _dev(kb), _dev(vb), grid, q_video, q_pos0, k_video, k_pos0, kv)
+    torch.cuda.synchronize()
+    assert H.last_device_error() == 0
+    q, k, v = (W.bf16_bits_to_f64(x) for x in (qb, kb, vb))
+    ref_o = np.empty((sq, heads, 128))
+    ref_l = np.empty((sq, heads))
+    for h in range(heads):
+        ref_o[:, h], ref_l[:, h] = O.joint_attention_block(q[0, :, h], k[0, :, h], v[0, :, h], grid, q_video, q_pos0,
+                                                           k_video, k_pos0, kv[0])
+    check(o[0].float().cpu().numpy().astype(np.float64), ref_o, "block out, no table")
+    check(lse[0].cpu().numpy().astype(np.float64), ref_l, "block lse, no table")
+    text_len, valid = 30, [12]
+    n = grid[0] * grid[1] * grid[2]
+    qw, kw, vw = (_dev(_bits((1, n + text_len, heads, 128), s)) for s in (14, 15, 16))
+    ref = H.attn_forward(qw, kw, vw, grid, text_len, valid)
+    whole, _ = H.attn_forward_block(qw, kw, vw, grid, n, 0, n, 0, [n + valid[0]], out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(whole, ref)
+
+
 def test_merge_kernel_matches_rule():
     rows = 1000
     rng = np.random.default_rng(4)
