@@ -517,7 +517,8 @@ def run_ours(args, wl, inp, rank, world, local):
                        "the step is a seconds-long loop of one kernel",
         "frac_of_burst": achieved / peak_burst, "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
         "algorithmic_flops_per_launch": flops,
-        "launch_ms": {"mean": mean_launch, "min": min(launch_ms), "max": max(launch_ms)},
+        "launch_ms": {"mean": mean_launch, "median": statistics.median(launch_ms), "min": min(launch_ms),
+                      "max": max(launch_ms), "count": len(launch_ms)},
     }
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
