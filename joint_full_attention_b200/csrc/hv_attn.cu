@@ -429,7 +429,12 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
     const uint32_t tab = table + 4u * static_cast<uint32_t>(L.table_base + L.i0);
     const int stride = 2 * L.half_dim;
     if constexpr (TABLE) {
-        // two rows (r, r + ROPE_GROUPS) per iteration so that their loads overlap
+        // two rows (r, r + ROPE_GROUPS) per iteration so that their loads overlap;
+        // the t and h lanes keep the (cos, sin) of their last position and read
+        // the table only when it changes (every Hp*Wp or Wp tokens)
+        const bool keep = L.axis != 2;
+        int kpos = -1;
+        uint4 kc = make_uint4(0u, 0u, 0u, 0u), ks = kc;
 #pragma unroll 1
         for (int r = rb; r < ROWS; r += 2 * ROPE_GROUPS) {
             const int pos0 = L.axis == 0 ? g.t : (L.axis == 1 ? g.h : g.w);
@@ -441,14 +446,22 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t table, int n0,
             const uint32_t t0 = tab + 4u * static_cast<uint32_t>(pos0 * stride);
             const uint32_t t1 = tab + 4u * static_cast<uint32_t>(pos1 * stride);
             const uint4 d0 = lds128(a0);
-            const uint4 c0 = lds128(t0);
-            const uint4 s0 = lds128(t0 + sin_off);
+            uint4 c0 = kc, s0 = ks;
+            if (!keep || pos0 != kpos) {
+                c0 = lds128(t0);
+                s0 = lds128(t0 + sin_off);
+            }
             uint4 d1 = d0, c1 = c0, s1 = s0;
             if (has1) {
                 d1 = lds128(a1);
-                c1 = lds128(t1);
-                s1 = lds128(t1 + sin_off);
+                if (!keep || pos1 != pos0) {
+                    c1 = lds128(t1);
+                    s1 = lds128(t1 + sin_off);
+                }
             }
+            kpos = has1 ? pos1 : pos0;
+            kc = has1 ? c1 : c0;
+            ks = has1 ? s1 : s0;
             sts128(a0, rotate_chunk(d0, c0, s0));
             if (!has1) break;
             sts128(a1, rotate_chunk(d1, c1, s1));
